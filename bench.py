@@ -1,0 +1,364 @@
+"""Benchmark of the routed-expert MoE layer on B200.
+
+Default workload: the GLM-scale decode layer (hidden 6144, expert intermediate
+2048, 256 routed + 1 shared int4 experts resident in HBM, top-8 of 8 groups /
+4 kept, routed_scaling_factor 2.5), one token per step with a fresh seed.  A
+step is one moe_layer_forward call: router logits + top-k, bucketing, expert
+gate/up + SwiGLU, down projection, combine.  Weight quantisation is load time
+and is reported separately.
+
+Timing: W warm-up steps, then K timed steps; L2 (126 MB) is flushed before each
+step by writing a 256 MB buffer outside the timed events; each step is timed
+with CUDA events on the launching stream; the job time is the max over ranks.
+With --gpus N > 1 every rank runs its own replica (the layer does not shard:
+no collective on the data path), so scaling is weak.
+
+--impl reference times the CPU oracle (test infrastructure) on the same
+workload, one token per step.
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import int4_routed_expert_route_b200 as lib  # noqa: E402
+from int4_routed_expert_route_b200 import synthetic as syn  # noqa: E402
+
+METRIC = "MoE-layer tokens/s and int4 expert-weight HBM GB/s (fraction of roofline) on 1 B200"
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.th = threading.Thread(target=self._read, daemon=True)
+            self.th.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [c.strip() for c in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def build_layer(cfg, layer=0, dev="cuda"):
+    experts = []
+    t0 = time.perf_counter()
+    qbytes = 0
+    for e in range(cfg.E + 1):
+        w = [syn.expert_weight(cfg, layer, e, m, dev) for m in ("gate", "up", "down")]
+        ex = lib.QuantExpert.from_fp32(*w, bits=cfg.bits)
+        qbytes += sum(x.numel() * 4 for x in w)
+        experts.append(ex)
+        del w
+    torch.cuda.synchronize()
+    load_s = time.perf_counter() - t0
+    table = lib.ExpertTable(experts[:cfg.E], dev)
+    shared = lib.SharedExpert(experts[cfg.E], dev)
+    gate = syn.router_gate(cfg, layer, dev)
+    bias = syn.router_bias(cfg, layer, dev)
+    rc = lib.router_cfg(cfg.E, cfg.k, cfg.n_group, cfg.topk_group, cfg.rsf, cfg.topp)
+    return dict(experts=experts, table=table, shared=shared, gate=gate, bias=bias, rc=rc,
+                load_s=load_s, fp32_bytes=qbytes,
+                expert_bytes=experts[0].nbytes())
+
+
+def run_ours(args, world, rank):
+    cfg = syn.DECODE
+    T = cfg.T
+    dev = torch.device("cuda")
+    L = build_layer(cfg)
+    stream = torch.cuda.current_stream()
+    K, W = args.steps, args.warmup
+    xs = syn.activations((K + W) * T, cfg.H, 1 + 1000003 * rank, dev).view(K + W, T, cfg.H)
+    y = torch.empty((T, cfg.H), dtype=torch.float32, device=dev)
+    ws = lib.Workspace(lib.moe_layer_workspace_bytes(T, cfg.H, cfg.I, L["rc"]), dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    nsteps = K + W
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(lib.LAYER_EVENTS)]
+          for _ in range(nsteps)]
+    for e in (x for row in ev for x in row):
+        e.record(stream)
+    torch.cuda.synchronize()
+
+    def step(i, events=None):
+        lib.moe_layer_forward(xs[i], L["gate"], L["bias"], L["rc"], L["table"], L["shared"],
+                              cfg.bits, y=y, ws=ws, events=events)
+
+    for i in range(W):
+        flush.fill_(i & 0xff)
+        step(i, ev[i])
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    clocks = ClockSampler(torch.cuda.current_device())
+    clocks.start()
+    time.sleep(0.3)
+    torch.cuda.synchronize()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for i in range(W, nsteps):
+        flush.fill_(i & 0xff)
+        step(i, ev[i])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    stage_ms = np.array([[ev[i][s].elapsed_time(ev[i][s + 1]) for s in range(lib.LAYER_EVENTS - 1)]
+                         for i in range(W, nsteps)])
+    step_ms = stage_ms.sum(axis=1)
+    total_ms = float(step_ms.sum())
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        total_ms = float(t.item())
+    clk = clocks.stop()
+
+    # end to end through the C ABI with host buffers: pinned x in, y out, per step
+    hx = xs.cpu().pin_memory()
+    hy = torch.empty((T, cfg.H), dtype=torch.float32).pin_memory()
+    dx = torch.empty((T, cfg.H), dtype=torch.bfloat16, device=dev)
+    e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(nsteps)]
+    for i in range(nsteps):
+        flush.fill_(i & 0xff)
+        e2e_ev[i][0].record(stream)
+        dx.copy_(hx[i], non_blocking=True)
+        lib.moe_layer_forward(dx, L["gate"], L["bias"], L["rc"], L["table"], L["shared"],
+                              cfg.bits, y=y, ws=ws)
+        hy.copy_(y, non_blocking=True)
+        e2e_ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = sum(a.elapsed_time(b) for a, b in e2e_ev[W:])
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    assert ws.flags() == 0
+
+    peaks, peak_kind = measured_peaks()
+    H, I = cfg.H, cfg.I
+    unique = cfg.k + 1  # T = 1: k distinct routed experts + the shared expert
+    gu_bytes = unique * 2 * (I * H // 2 + I * 4)        # gate + up nibbles and scales
+    dn_bytes = unique * (H * I // 2 + H * 4)
+    expert_bytes_step = gu_bytes + dn_bytes
+    gu_ms = float(np.mean(stage_ms[:, 2]))
+    achieved = gu_bytes / (gu_ms * 1e-3) / 1e9
+    tokens = K * T * world
+    value = tokens / (total_ms * 1e-3)
+    res = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": W,
+        "ms_per_step": round(total_ms / K, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "int4 weights, fp32 accumulate (bf16 activations)",
+        "data": "synthetic (seeded N(0,0.02) weights quantised on device; x ~ N(0,1) bf16)",
+        "config": {"workload": "GLM-scale MoE layer decode, T=1 per step, H=6144 I=2048 "
+                               "E=256+1 shared top-8 n_group=8 topk_group=4 rsf=2.5 int4",
+                   "tokens_per_step": T, "l2": "flushed before every step (256 MB write, "
+                                                "outside the timed events)",
+                   "parallelism": f"replicas x{world}"},
+        "expert_gbs": round(expert_bytes_step / (total_ms / K * 1e-3) / 1e9, 1),
+        "expert_bytes_per_token": expert_bytes_step,
+        "stage_ms_median": {n: round(float(np.median(stage_ms[:, s])), 5) for s, n in
+                            enumerate(["router", "bucket", "gate_up", "down", "combine"])},
+        "roofline": {"kernel": "gateup_gemv (int4 gate+up GEMV + SwiGLU)", "bound": "hbm",
+                     "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
+                     "peak_source": peak_kind, "unit": "GB/s",
+                     "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": None,
+                     "algorithmic_bytes_per_launch": gu_bytes},
+        "e2e": {"value": round(tokens / (e2e_ms * 1e-3), 2), "unit": "tokens/s",
+                "h2d_bytes_per_step": T * H * 2, "d2h_bytes_per_step": T * H * 4},
+        "gpu_launches": 6 * K,
+        "clocks": clk,
+        "load": {"quantize_s": round(L["load_s"], 3), "fp32_bytes": L["fp32_bytes"],
+                 "int4_expert_bytes": L["expert_bytes"]},
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = cpu_baseline(cfg, L, xs[W:W + 2], samples=1)
+    return res
+
+
+def _oracle_expert(orc, cfg, e, dev="cuda"):
+    w = [syn.expert_weight(cfg, 0, e, m, dev).cpu().numpy() for m in ("gate", "up", "down")]
+    q = [orc.quantize_rows(wi, cfg.bits) for wi in w]
+    return orc.Expert(q[0][0], q[0][1], q[1][0], q[1][1], q[2][0], q[2][1], cfg.bits)
+
+
+def cpu_baseline(cfg, L, xs, samples=1):
+    """The oracle timed on the host cores on `samples` tokens of the workload."""
+    import oracle as orc
+    gate = L["gate"].cpu().numpy()
+    bias = L["bias"].cpu().numpy()
+    xb = syn.bf16_bits(xs.reshape(-1, cfg.H)[:samples])
+    r = orc.route(xb, gate, bias, cfg.k, cfg.n_group, cfg.topk_group, cfg.rsf)
+    need = sorted(set(int(e) for e in r["idx"].reshape(-1)))
+    experts = [_oracle_expert(orc, cfg, e) if e in need else None for e in range(cfg.E)]
+    shared = _oracle_expert(orc, cfg, cfg.E)
+    t0 = time.perf_counter()
+    orc.layer(xb, gate, bias, experts, shared, cfg.H, cfg.I, cfg.k, cfg.n_group,
+              cfg.topk_group, cfg.rsf)
+    dt = time.perf_counter() - t0
+    return {"value": round(samples / dt, 4), "unit": "tokens/s", "cores": orc.num_threads(),
+            "kind": "oracle",
+            "sample": f"{samples} token(s) of the GLM-scale decode layer through the fp64 C "
+                      f"oracle (routing + 9 experts), experts quantised beforehand (untimed)"}
+
+
+def run_reference(args, world, rank):
+    import oracle as orc
+    cfg = syn.DECODE
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    gate = syn.router_gate(cfg, 0, dev).cpu().numpy()
+    bias = syn.router_bias(cfg, 0, dev).cpu().numpy()
+    K, W = args.steps, args.warmup
+    xs = syn.bf16_bits(syn.activations(K + W, cfg.H, 1, dev))
+    cache = {}
+
+    def expert(e):
+        if e not in cache:
+            cache[e] = _oracle_expert(orc, cfg, e, dev)
+        return cache[e]
+
+    def step(i):
+        r = orc.route(xs[i:i + 1], gate, bias, cfg.k, cfg.n_group, cfg.topk_group, cfg.rsf)
+        experts = [None] * cfg.E
+        for e in r["idx"].reshape(-1):
+            experts[int(e)] = expert(int(e))
+        return experts, r
+
+    sh = expert(cfg.E)
+    times = []
+    for i in range(K + W):
+        experts, r = step(i)  # expert preparation (quantisation) is load time, untimed
+        t0 = time.perf_counter()
+        orc.layer(xs[i:i + 1], gate, bias, experts, sh, cfg.H, cfg.I, cfg.k, cfg.n_group,
+                  cfg.topk_group, cfg.rsf)
+        dt = time.perf_counter() - t0
+        if i >= W:
+            times.append(dt)
+    total = sum(times)
+    value = K / total
+    return {
+        "impl": "reference",
+        "metric": METRIC, "value": round(value, 4), "unit": "tokens/s", "n_gpus": 1,
+        "steps": K, "warmup": W, "ms_per_step": round(total / K * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": "GLM-scale MoE layer decode, T=1 per step, H=6144 I=2048 "
+                               "E=256+1 shared top-8 n_group=8 topk_group=4 rsf=2.5 int4",
+                   "tokens_per_step": 1},
+        "cpu_baseline": {"value": round(value, 4), "unit": "tokens/s", "cores": orc.num_threads(),
+                         "kind": "oracle",
+                         "sample": "one token per step through the fp64 C oracle layer "
+                                   "(routing + 9 experts); expert quantisation untimed"},
+        "e2e": {"value": round(value, 4), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        if rank != 0:
+            return
+        print(json.dumps(run_reference(args, 1, 0)))
+        return
+    lib.load()
+    world, rank, _ = dist_setup()
+    res = run_ours(args, world, rank)
+    if rank == 0:
+        print(json.dumps(res))
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

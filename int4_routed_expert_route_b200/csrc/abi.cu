@@ -1,0 +1,300 @@
+// abi.cu -- the extern "C" entry points of include/moe.h: argument checks,
+// workspace layout and the kernel sequence of each call.  Nothing here
+// allocates device memory; all scratch lives in the caller's workspace.
+#include <cstring>
+
+#include "common.cuh"
+
+namespace moe {
+
+// Kernel launchers (one per translation unit).
+moe_status launch_quantize(const float *, int64_t, int64_t, int32_t, uint8_t *, float *, cudaStream_t);
+moe_status launch_route(const uint16_t *, int64_t, int64_t, const float *, const float *,
+                        const moe_router_cfg *, int32_t *, float *, float *, double *, cudaStream_t);
+size_t route_part_bytes(int64_t T, int64_t H, int E);
+int route_ks_for(int64_t T, int64_t H);
+moe_status launch_bucket(const int32_t *, int64_t, int32_t, int32_t, int32_t *, int32_t *, int32_t *,
+                         int32_t *, int32_t *, int32_t *, int32_t *, uint32_t *, int32_t, int32_t *,
+                         cudaStream_t);
+struct GemvArgs;
+moe_status launch_combine(float *, const float *, const int32_t *, const float *, int64_t, int64_t,
+                          int32_t, bool, bool, cudaStream_t);
+moe_status launch_rmsnorm(const float *, int64_t, int64_t, float, uint16_t *, cudaStream_t);
+moe_status run_gemv_layer(const uint16_t *x, int64_t T, int64_t H, int64_t I, int32_t k, int32_t bits,
+                          const moe_expert *experts, const moe_expert *shared, const int32_t *unique,
+                          const int32_t *n_unique, const int32_t *offsets, const int32_t *tok,
+                          float *h, float *yp, uint32_t *flags, int64_t max_segments,
+                          int64_t max_tok, cudaStream_t stream, cudaEvent_t ev_down);
+moe_status run_gemv_single(const uint16_t *x, int64_t T, int64_t H, int64_t I, const moe_expert &e,
+                           const int32_t *rows, const float *row_w, int64_t n_rows, float *h,
+                           float *y, uint32_t *flags, cudaStream_t stream);
+
+static constexpr size_t kAlign = 256;
+static size_t up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
+
+static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+static bool cfg_ok(const moe_router_cfg *c) {
+    if (!c) return false;
+    const int E = c->n_experts, k = c->top_k, ng = c->n_group, tkg = c->topk_group;
+    if (E < 1 || E > 1024 || k < 1 || k > 32 || ng < 1 || ng > 32 || tkg < 1) return false;
+    if (E % ng || tkg > ng) return false;
+    if (ng > 1 && E / ng < 2) return false;
+    if (k > tkg * (E / ng)) return false;
+    if (!(c->routed_scaling_factor == c->routed_scaling_factor)) return false;
+    if (!(c->expert_topp >= 0.0f)) return false;
+    return true;
+}
+
+// Largest batch the CUDA-core path takes on; larger batches use tensor cores.
+static constexpr int64_t kGemvMaxT = 4096;
+
+bool plan_layer(int64_t T, int64_t H, int64_t I, const moe_router_cfg *cfg, int32_t path,
+                LayerPlan *p) {
+    if (!cfg_ok(cfg) || T < 0 || H <= 0 || I <= 0) return false;
+    std::memset(p, 0, sizeof(*p));
+    p->T = T;
+    p->H = H;
+    p->I = I;
+    p->E = cfg->n_experts;
+    p->k = cfg->top_k;
+    p->path = path == MOE_PATH_AUTO ? MOE_PATH_GEMV : path;
+    p->route_ks = route_ks_for(T, H);
+    const size_t P = static_cast<size_t>(T) * p->k;
+    const size_t E = static_cast<size_t>(p->E);
+    const size_t Pall = P + static_cast<size_t>(T);
+    size_t o = 0;
+    p->off_flags = o;   o = up(o + 256);
+    p->off_part = o;    o = up(o + route_part_bytes(T, H, p->E));
+    p->off_idx = o;     o = up(o + P * 4);
+    p->off_w = o;       o = up(o + P * 4);
+    p->off_counts = o;  o = up(o + E * 4);
+    p->off_offsets = o; o = up(o + (E + 1) * 4);
+    p->off_list = o;    o = up(o + P * 4);
+    p->off_tok = o;     o = up(o + P * 4);
+    p->off_pos = o;     o = up(o + P * 4);
+    p->off_unique = o;  o = up(o + E * 4);
+    p->off_nunique = o; o = up(o + 4);
+    p->off_tiles = o;   o = up(o + (E + 2) * 4);
+    p->off_h = o;       o = up(o + Pall * static_cast<size_t>(I) * 4);
+    p->off_yp = o;      o = up(o + Pall * static_cast<size_t>(H) * 4);
+    p->total = o;
+    return true;
+}
+
+}  // namespace moe
+
+using namespace moe;
+
+#define CUDA_OK(x) ((x) == cudaSuccess)
+
+extern "C" {
+
+const char *moe_status_str(moe_status s) {
+    switch (s) {
+    case MOE_OK: return "MOE_OK";
+    case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG";
+    case MOE_ERR_UNSUPPORTED: return "MOE_ERR_UNSUPPORTED";
+    case MOE_ERR_CUDA: return "MOE_ERR_CUDA";
+    case MOE_ERR_WORKSPACE: return "MOE_ERR_WORKSPACE";
+    case MOE_ERR_DEVICE_FLAG: return "MOE_ERR_DEVICE_FLAG";
+    }
+    return "MOE_STATUS_UNKNOWN";
+}
+
+int32_t moe_abi_version(void) { return 1; }
+
+moe_status moe_workspace_init(void *ws, size_t ws_bytes, cudaStream_t stream) {
+    if (!ws || ws_bytes < 256) return MOE_ERR_WORKSPACE;
+    return CUDA_OK(cudaMemsetAsync(ws, 0, 256, stream)) ? MOE_OK : MOE_ERR_CUDA;
+}
+
+moe_status moe_workspace_status(const void *ws, cudaStream_t stream, uint32_t *flags_out) {
+    if (!ws) return MOE_ERR_WORKSPACE;
+    uint32_t f = 0;
+    if (!CUDA_OK(cudaStreamSynchronize(stream))) return MOE_ERR_CUDA;
+    if (!CUDA_OK(cudaMemcpy(&f, ws, sizeof(f), cudaMemcpyDeviceToHost))) return MOE_ERR_CUDA;
+    if (flags_out) *flags_out = f;
+    return f ? MOE_ERR_DEVICE_FLAG : MOE_OK;
+}
+
+moe_status moe_quantize_rows(const float *w, int64_t rows, int64_t cols, int32_t bits,
+                             uint8_t *q_out, float *scale_out, cudaStream_t stream) {
+    if (rows < 0 || cols <= 0) return MOE_ERR_INVALID_ARG;
+    if (bits != 2 && bits != 4 && bits != 8) return MOE_ERR_INVALID_ARG;
+    if ((bits == 4 && cols % 2) || (bits == 2 && cols % 4)) return MOE_ERR_INVALID_ARG;
+    if (rows > 0 && (!w || !q_out || !scale_out)) return MOE_ERR_INVALID_ARG;
+    return launch_quantize(w, rows, cols, bits, q_out, scale_out, stream);
+}
+
+size_t moe_route_workspace_bytes(int64_t T, int64_t H, const moe_router_cfg *cfg) {
+    if (!cfg_ok(cfg) || T < 0 || H <= 0) return 0;
+    return 256 + up(route_part_bytes(T, H, cfg->n_experts));
+}
+
+moe_status moe_route_topk(const uint16_t *x, int64_t T, int64_t H, const float *gate,
+                          const float *bias, const moe_router_cfg *cfg, int32_t *idx_out,
+                          float *w_out, float *gap_out, void *ws, size_t ws_bytes,
+                          cudaStream_t stream) {
+    if (!cfg_ok(cfg) || T < 0 || H <= 0 || H % 64) return MOE_ERR_INVALID_ARG;
+    if (T > 0 && (!x || !gate || !bias || !idx_out || !w_out)) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(gate)) return MOE_ERR_INVALID_ARG;
+    const size_t need = moe_route_workspace_bytes(T, H, cfg);
+    if (!ws || ws_bytes < need || !aligned16(ws)) return MOE_ERR_WORKSPACE;
+    double *part = reinterpret_cast<double *>(static_cast<char *>(ws) + 256);
+    return launch_route(x, T, H, gate, bias, cfg, idx_out, w_out, gap_out, part, stream);
+}
+
+moe_status moe_bucket(const int32_t *idx, int64_t T, int32_t k, int32_t E, int32_t *counts,
+                      int32_t *offsets, int32_t *list, int32_t *unique, int32_t *n_unique,
+                      cudaStream_t stream) {
+    if (T < 0 || k < 1 || E < 1 || E > 1024 || T * k > (1ll << 24)) return MOE_ERR_INVALID_ARG;
+    if ((T > 0 && !idx) || !counts || !offsets || !unique || !n_unique) return MOE_ERR_INVALID_ARG;
+    if (T > 0 && !list) return MOE_ERR_INVALID_ARG;
+    return launch_bucket(idx, T, k, E, counts, offsets, list, nullptr, nullptr, unique, n_unique,
+                         nullptr, 0, nullptr, stream);
+}
+
+static bool qmat_host_ok(const moe_qmat &m, int64_t rows, int64_t cols) {
+    return m.q && m.scale && (m.bits == 2 || m.bits == 4 || m.bits == 8) && m.reserved == 0 &&
+           m.rows == rows && m.cols == cols && aligned16(m.q);
+}
+
+size_t moe_expert_ffn_workspace_bytes(int64_t n_rows, int64_t H, int64_t I) {
+    if (n_rows < 0 || H <= 0 || I <= 0) return 0;
+    return 256 + up(static_cast<size_t>(n_rows) * static_cast<size_t>(I) * 4);
+}
+
+moe_status moe_expert_ffn(const uint16_t *x, int64_t T, int64_t H, int64_t I,
+                          const moe_expert *e, const int32_t *rows, const float *row_w,
+                          int64_t n_rows, float *y, void *ws, size_t ws_bytes,
+                          cudaStream_t stream) {
+    if (T < 0 || H <= 0 || I <= 0 || H % 64 || I % 64 || !e) return MOE_ERR_INVALID_ARG;
+    if (!rows) n_rows = T;
+    if (n_rows < 0 || (rows == nullptr && n_rows != T)) return MOE_ERR_INVALID_ARG;
+    if (n_rows > 0 && (!x || !y)) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(y)) return MOE_ERR_INVALID_ARG;
+    if (!qmat_host_ok(e->gate, I, H) || !qmat_host_ok(e->up, I, H) || !qmat_host_ok(e->down, H, I))
+        return MOE_ERR_INVALID_ARG;
+    if (e->gate.bits != e->up.bits || e->gate.bits != e->down.bits) return MOE_ERR_INVALID_ARG;
+    const size_t need = moe_expert_ffn_workspace_bytes(n_rows, H, I);
+    if (!ws || ws_bytes < need || !aligned16(ws)) return MOE_ERR_WORKSPACE;
+    if (n_rows == 0) return MOE_OK;
+    float *h = reinterpret_cast<float *>(static_cast<char *>(ws) + 256);
+    return run_gemv_single(x, T, H, I, *e, rows, row_w, n_rows, h, y,
+                           static_cast<uint32_t *>(ws), stream);
+}
+
+size_t moe_layer_workspace_bytes(int64_t T, int64_t H, int64_t I, const moe_router_cfg *cfg) {
+    LayerPlan p;
+    if (!plan_layer(T, H, I, cfg, MOE_PATH_AUTO, &p)) return 0;
+    return p.total;
+}
+
+static void rec(cudaEvent_t *ev, int i, cudaStream_t s) {
+    if (ev && ev[i]) cudaEventRecord(ev[i], s);
+}
+
+moe_status moe_layer_forward_ex(const uint16_t *x, int64_t T, int64_t H, int64_t I,
+                                const float *gate, const float *bias, const moe_router_cfg *cfg,
+                                const moe_expert *experts, const moe_expert *shared,
+                                int32_t weight_bits, float *y, int32_t *idx_out, float *w_out,
+                                void *ws, size_t ws_bytes, int32_t path, int32_t accumulate,
+                                cudaEvent_t *events, cudaStream_t stream) {
+    if (!cfg_ok(cfg) || T < 0 || H <= 0 || I <= 0 || H % 64 || I % 64) return MOE_ERR_INVALID_ARG;
+    if (weight_bits != 2 && weight_bits != 4 && weight_bits != 8) return MOE_ERR_INVALID_ARG;
+    if (path != MOE_PATH_AUTO && path != MOE_PATH_GEMV && path != MOE_PATH_TENSOR)
+        return MOE_ERR_INVALID_ARG;
+    if (T > 0 && (!x || !gate || !bias || !experts || !y)) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(gate) || !aligned16(y) || !aligned16(experts))
+        return MOE_ERR_INVALID_ARG;
+    LayerPlan p;
+    if (!plan_layer(T, H, I, cfg, path, &p)) return MOE_ERR_INVALID_ARG;
+    if (p.path == MOE_PATH_TENSOR) return MOE_ERR_UNSUPPORTED;
+    if (p.path == MOE_PATH_GEMV && T > kGemvMaxT) return MOE_ERR_UNSUPPORTED;
+    if (!ws || ws_bytes < p.total || !aligned16(ws)) return MOE_ERR_WORKSPACE;
+    if (T == 0) return MOE_OK;
+    char *base = static_cast<char *>(ws);
+    uint32_t *flags = reinterpret_cast<uint32_t *>(base + p.off_flags);
+    int32_t *idx = idx_out ? idx_out : reinterpret_cast<int32_t *>(base + p.off_idx);
+    float *w = w_out ? w_out : reinterpret_cast<float *>(base + p.off_w);
+    int32_t *counts = reinterpret_cast<int32_t *>(base + p.off_counts);
+    int32_t *offsets = reinterpret_cast<int32_t *>(base + p.off_offsets);
+    int32_t *list = reinterpret_cast<int32_t *>(base + p.off_list);
+    int32_t *tok = reinterpret_cast<int32_t *>(base + p.off_tok);
+    int32_t *pos = reinterpret_cast<int32_t *>(base + p.off_pos);
+    int32_t *unique = reinterpret_cast<int32_t *>(base + p.off_unique);
+    int32_t *nunique = reinterpret_cast<int32_t *>(base + p.off_nunique);
+    float *h = reinterpret_cast<float *>(base + p.off_h);
+    float *yp = reinterpret_cast<float *>(base + p.off_yp);
+    moe_status st;
+
+    rec(events, 0, stream);
+    st = launch_route(x, T, H, gate, bias, cfg, idx, w, nullptr,
+                      reinterpret_cast<double *>(base + p.off_part), stream);
+    if (st != MOE_OK) return st;
+    rec(events, 1, stream);
+    st = launch_bucket(idx, T, p.k, p.E, counts, offsets, list, tok, pos, unique, nunique, flags, 0,
+                       nullptr, stream);
+    if (st != MOE_OK) return st;
+    rec(events, 2, stream);
+    const int64_t max_seg = (T * p.k < p.E ? T * p.k : p.E) + (shared ? 1 : 0);
+    const int64_t max_tok = T;
+    st = run_gemv_layer(x, T, H, I, p.k, weight_bits, experts, shared, unique, nunique, offsets, tok, h, yp,
+                        flags, max_seg, max_tok, stream, events ? events[3] : nullptr);
+    if (st != MOE_OK) return st;
+    rec(events, 4, stream);
+    st = launch_combine(y, yp, pos, w, T, H, p.k, shared != nullptr, accumulate != 0, stream);
+    if (st != MOE_OK) return st;
+    rec(events, 5, stream);
+    return MOE_OK;
+}
+
+moe_status moe_layer_forward(const uint16_t *x, int64_t T, int64_t H, int64_t I,
+                             const float *gate, const float *bias, const moe_router_cfg *cfg,
+                             const moe_expert *experts, const moe_expert *shared,
+                             int32_t weight_bits, float *y, int32_t *idx_out, float *w_out,
+                             void *ws, size_t ws_bytes, cudaStream_t stream) {
+    return moe_layer_forward_ex(x, T, H, I, gate, bias, cfg, experts, shared, weight_bits, y,
+                                idx_out, w_out, ws, ws_bytes, MOE_PATH_AUTO, 0, nullptr, stream);
+}
+
+moe_status moe_rmsnorm_bf16(const float *v, int64_t T, int64_t H, float eps, uint16_t *out,
+                            cudaStream_t stream) {
+    if (T < 0 || H <= 0 || (T > 0 && (!v || !out)) || !(eps >= 0.0f)) return MOE_ERR_INVALID_ARG;
+    return launch_rmsnorm(v, T, H, eps, out, stream);
+}
+
+size_t moe_stack_workspace_bytes(int64_t T, int64_t H, int64_t I, const moe_router_cfg *cfg) {
+    const size_t l = moe_layer_workspace_bytes(T, H, I, cfg);
+    if (!l) return 0;
+    return l + up(static_cast<size_t>(T) * static_cast<size_t>(H) * 2);
+}
+
+moe_status moe_stack_forward(float *resid, int64_t T, int64_t H, int64_t I, int32_t n_layers,
+                             const moe_layer_params *layers, const moe_router_cfg *cfg,
+                             float eps, uint16_t *layer_inputs, int32_t *idx_out, void *ws,
+                             size_t ws_bytes, cudaStream_t stream) {
+    if (n_layers < 0 || (n_layers > 0 && !layers) || !cfg_ok(cfg)) return MOE_ERR_INVALID_ARG;
+    if (T > 0 && !resid) return MOE_ERR_INVALID_ARG;
+    const size_t lw = moe_layer_workspace_bytes(T, H, I, cfg);
+    const size_t need = moe_stack_workspace_bytes(T, H, I, cfg);
+    if (!lw || !ws || ws_bytes < need || !aligned16(ws)) return MOE_ERR_WORKSPACE;
+    if (T == 0) return MOE_OK;
+    uint16_t *xin_ws = reinterpret_cast<uint16_t *>(static_cast<char *>(ws) + lw);
+    const int64_t k = cfg->top_k;
+    for (int32_t l = 0; l < n_layers; l++) {
+        uint16_t *xin = layer_inputs ? layer_inputs + static_cast<int64_t>(l) * T * H : xin_ws;
+        moe_status st = launch_rmsnorm(resid, T, H, eps, xin, stream);
+        if (st != MOE_OK) return st;
+        st = moe_layer_forward_ex(xin, T, H, I, layers[l].gate, layers[l].bias, cfg,
+                                  layers[l].experts, layers[l].shared, layers[l].weight_bits,
+                                  resid,
+                                  idx_out ? idx_out + static_cast<int64_t>(l) * T * k : nullptr,
+                                  nullptr, ws, lw, MOE_PATH_AUTO, 1, nullptr, stream);
+        if (st != MOE_OK) return st;
+    }
+    return MOE_OK;
+}
+
+}  // extern "C"

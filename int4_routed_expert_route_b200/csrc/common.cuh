@@ -1,0 +1,107 @@
+// common.cuh -- shared device helpers and the internal launch descriptors of
+// the MoE layer library (sm_100a).
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include "../../include/moe.h"
+
+namespace moe {
+
+constexpr int kWarp = 32;
+
+// ----------------------------------------------------------------------------
+// Device flag word (first 4 bytes of every workspace).
+// ----------------------------------------------------------------------------
+__device__ __forceinline__ void raise_flag(uint32_t *flags, uint32_t bit) {
+    if (flags) atomicOr(flags, bit);
+}
+
+// ----------------------------------------------------------------------------
+// Small arithmetic helpers.
+// ----------------------------------------------------------------------------
+__device__ __forceinline__ float bf16_bits_to_float(uint16_t b) {
+    return __uint_as_float(static_cast<uint32_t>(b) << 16);
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+__device__ __forceinline__ double warp_sum(double v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+
+// Packed pair of fp32 values in one 64-bit register (the sm_100 f32x2 datapath).
+struct f2 {
+    unsigned long long v;
+};
+
+__device__ __forceinline__ f2 f2_make(float lo, float hi) {
+    f2 r;
+    r.v = (static_cast<unsigned long long>(__float_as_uint(hi)) << 32) | __float_as_uint(lo);
+    return r;
+}
+__device__ __forceinline__ float f2_lo(f2 a) { return __uint_as_float(static_cast<uint32_t>(a.v)); }
+__device__ __forceinline__ float f2_hi(f2 a) { return __uint_as_float(static_cast<uint32_t>(a.v >> 32)); }
+
+// acc += a * b  (two lanes, round-to-nearest, no contraction surprises)
+__device__ __forceinline__ void f2_fma(f2 &acc, f2 a, f2 b) {
+    asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(acc.v) : "l"(a.v), "l"(b.v));
+}
+// a - b
+__device__ __forceinline__ f2 f2_sub(f2 a, f2 b) {
+    f2 r;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r.v) : "l"(a.v), "l"(b.v));
+    return r;
+}
+
+__device__ __forceinline__ float silu(float g) { return g / (1.0f + expf(-g)); }
+
+// 128-bit streaming load that does not allocate in L1 (weights are read once).
+__device__ __forceinline__ uint4 ldg_stream(const void *p) {
+    uint4 r;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+                 : "l"(p));
+    return r;
+}
+__device__ __forceinline__ uint2 ldg_stream8(const void *p) {
+    uint2 r;
+    asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];"
+                 : "=r"(r.x), "=r"(r.y)
+                 : "l"(p));
+    return r;
+}
+
+// ----------------------------------------------------------------------------
+// Workspace layout of one layer call (host computes, kernels receive pointers).
+// ----------------------------------------------------------------------------
+struct LayerPlan {
+    int64_t T, H, I;
+    int32_t E, k;
+    int32_t path;      // MOE_PATH_GEMV or MOE_PATH_TENSOR
+    int32_t route_ks;  // K-splits of the router logits
+    size_t off_flags, off_part, off_idx, off_w, off_counts, off_offsets, off_list, off_tok,
+        off_pos, off_unique, off_nunique, off_tiles, off_h, off_yp, total;
+};
+
+// Host: fills the plan for a layer call; returns false on an impossible size.
+bool plan_layer(int64_t T, int64_t H, int64_t I, const moe_router_cfg *cfg, int32_t path,
+                LayerPlan *p);
+
+}  // namespace moe
