@@ -162,6 +162,27 @@ MOE_API moe_status moe_route_topk(const uint16_t *x, int64_t T, int64_t H, const
                           cudaStream_t stream);
 
 /*
+ * moe_route_topk without a workspace, for callers that cannot allocate device
+ * memory when they route (a fixed, pre-planned memory budget; code that must not
+ * call an allocator because it may synchronise the device; a host that only holds
+ * raw device pointers from another runtime).  The pages have no counterpart: this
+ * is an interface convenience, with the same results as moe_route_topk.
+ * Scratch comes from a 4 MiB array inside the library, present on every GPU that
+ * loads the library until the process exits (moe_route_noalloc_max_scratch_bytes
+ * returns its size).  A request whose scratch, moe_route_workspace_bytes(T, H, cfg)
+ * minus 256, exceeds it returns MOE_ERR_WORKSPACE before anything is launched
+ * (GLM sizes: up to T = 64 on the small-batch kernels, T = 2048 above).
+ * The first call on a device looks up the array's address (make it before any
+ * stream capture).  All calls share the array: calls that overlap on the GPU race
+ * and must be serialised by the caller.  Allocates nothing.
+ */
+MOE_API size_t moe_route_noalloc_max_scratch_bytes(void);
+MOE_API moe_status moe_route_topk_noalloc(const uint16_t *x, int64_t T, int64_t H,
+                                          const float *gate, const float *bias,
+                                          const moe_router_cfg *cfg, int32_t *idx_out,
+                                          float *w_out, float *gap_out, cudaStream_t stream);
+
+/*
  * Batch-union bucketing ("Show HN", implemented features: each unique expert
  * of a batch is read once and applied to every position routed to it).
  * A stable counting sort of the (token, slot) pairs p = t*k + slot by expert:

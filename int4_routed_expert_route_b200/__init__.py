@@ -28,7 +28,8 @@ EXPORTS = ["moe_status_str", "moe_abi_version", "moe_workspace_init", "moe_works
            "moe_quantize_rows", "moe_route_workspace_bytes", "moe_route_topk", "moe_bucket",
            "moe_expert_ffn_workspace_bytes", "moe_expert_ffn", "moe_layer_workspace_bytes",
            "moe_layer_forward", "moe_layer_forward_ex", "moe_rmsnorm_bf16",
-           "moe_stack_workspace_bytes", "moe_stack_forward"]
+           "moe_stack_workspace_bytes", "moe_stack_forward",
+           "moe_route_noalloc_max_scratch_bytes", "moe_route_topk_noalloc"]
 
 
 class MoEError(RuntimeError):
@@ -77,7 +78,8 @@ def load():
     L.moe_status_str.restype = ctypes.c_char_p
     L.moe_abi_version.restype = _i32
     for name in ("moe_route_workspace_bytes", "moe_expert_ffn_workspace_bytes",
-                 "moe_layer_workspace_bytes", "moe_stack_workspace_bytes"):
+                 "moe_layer_workspace_bytes", "moe_stack_workspace_bytes",
+                 "moe_route_noalloc_max_scratch_bytes"):
         getattr(L, name).restype = _sz
     L.moe_route_workspace_bytes.argtypes = [_i64, _i64, ctypes.POINTER(moe_router_cfg)]
     L.moe_expert_ffn_workspace_bytes.argtypes = [_i64, _i64, _i64]
@@ -92,6 +94,9 @@ def load():
     L.moe_quantize_rows.argtypes = [_vp, _i64, _i64, _i32, _vp, _vp, _vp]
     L.moe_route_topk.argtypes = [_vp, _i64, _i64, _vp, _vp, ctypes.POINTER(moe_router_cfg), _vp,
                                  _vp, _vp, _vp, _sz, _vp]
+    L.moe_route_noalloc_max_scratch_bytes.argtypes = []
+    L.moe_route_topk_noalloc.argtypes = [_vp, _i64, _i64, _vp, _vp,
+                                         ctypes.POINTER(moe_router_cfg), _vp, _vp, _vp, _vp]
     L.moe_bucket.argtypes = [_vp, _i64, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _vp]
     L.moe_expert_ffn.argtypes = [_vp, _i64, _i64, _i64, ctypes.POINTER(moe_expert), _vp, _vp,
                                  _i64, _vp, _vp, _sz, _vp]
@@ -239,6 +244,22 @@ def moe_route_topk(x, gate, bias, cfg, ws=None, with_gap=False, stream=None):
                                                    ctypes.byref(cfg), _ptr(idx), _ptr(w),
                                                    _ptr(gap), ws.ptr(), ws.nbytes,
                                                    _stream(stream)))
+    return idx, w, gap
+
+
+def moe_route_topk_noalloc(x, gate, bias, cfg, with_gap=False, stream=None):
+    """moe_route_topk with the library's built-in scratch (no workspace)."""
+    x = _bf16(x, "x")
+    gate = _dev(gate, torch.float32, "gate")
+    bias = _dev(bias, torch.float32, "bias")
+    T, H = x.shape
+    k = cfg.top_k
+    idx = torch.empty((T, k), dtype=torch.int32, device=x.device)
+    w = torch.empty((T, k), dtype=torch.float32, device=x.device)
+    gap = torch.empty(T, dtype=torch.float32, device=x.device) if with_gap else None
+    _check("moe_route_topk_noalloc", load().moe_route_topk_noalloc(
+        _ptr(x), T, H, _ptr(gate), _ptr(bias), ctypes.byref(cfg), _ptr(idx), _ptr(w), _ptr(gap),
+        _stream(stream)))
     return idx, w, gap
 
 
