@@ -112,8 +112,10 @@ MOE_API const char *moe_status_str(moe_status s);
 MOE_API int32_t moe_abi_version(void);
 
 /*
- * Clear the device flag word at the start of a workspace (async on stream).
- * Call once on a fresh workspace and after reading a latched flag.
+ * Clear the header of a workspace (its first 4 KiB, or ws_bytes if smaller:
+ * the device flag word and the counters the layer kernels keep between calls),
+ * async on stream.  Call once on a fresh workspace and after reading a latched
+ * flag.
  */
 MOE_API moe_status moe_workspace_init(void *ws, size_t ws_bytes, cudaStream_t stream);
 
@@ -171,7 +173,7 @@ MOE_API moe_status moe_route_topk(const uint16_t *x, int64_t T, int64_t H, const
  * loads the library until the process exits (moe_route_noalloc_max_scratch_bytes
  * returns its size).  A request whose scratch, moe_route_workspace_bytes(T, H, cfg)
  * minus 256, exceeds it returns MOE_ERR_WORKSPACE before anything is launched
- * (GLM sizes: up to T = 64 on the small-batch kernels, T = 2048 above).
+ * (the scratch is T * n_experts fp32 logits: up to T = 4096 with 256 experts).
  * The first call on a device looks up the array's address (make it before any
  * stream capture).  All calls share the array: calls that overlap on the GPU race
  * and must be serialised by the caller.  Allocates nothing.

@@ -20,6 +20,19 @@ struct GemvArgs;
 moe_status launch_combine(float *, const float *, const int32_t *, const float *, int64_t, int64_t,
                           int32_t, bool, bool, cudaStream_t);
 moe_status launch_rmsnorm(const float *, int64_t, int64_t, float, uint16_t *, cudaStream_t);
+bool route_fused_ok(int64_t T, int64_t H);
+moe_status launch_route_fused(const uint16_t *, int64_t, int64_t, const float *, const float *,
+                              const moe_router_cfg *, int32_t *, float *, float *, unsigned *,
+                              int32_t *, int32_t *, int32_t *, int32_t *, int32_t *, int32_t *,
+                              int32_t *, uint32_t *, int32_t *, int32_t, cudaStream_t);
+bool decode_ok(int64_t T, int64_t H, int64_t I, int32_t k, int32_t bits);
+moe_status run_decode_layer(const uint16_t *x, int64_t T, int64_t H, int64_t I, int32_t k,
+                            int32_t bits, const moe_expert *experts, const moe_expert *shared,
+                            const int32_t *unique, const int32_t *n_unique, const int32_t *offsets,
+                            const int32_t *tok, const int32_t *pos, const int32_t *idx,
+                            const float *w, float *h, float *yp, int32_t *tile_cnt, float *y,
+                            int32_t accumulate, uint32_t *flags, cudaStream_t stream,
+                            cudaEvent_t ev_down);
 moe_status run_gemv_layer(const uint16_t *x, int64_t T, int64_t H, int64_t I, int32_t k, int32_t bits,
                           const moe_expert *experts, const moe_expert *shared, const int32_t *unique,
                           const int32_t *n_unique, const int32_t *offsets, const int32_t *tok,
@@ -30,6 +43,9 @@ moe_status run_gemv_single(const uint16_t *x, int64_t T, int64_t H, int64_t I, c
                            float *y, uint32_t *flags, cudaStream_t stream);
 
 static constexpr size_t kAlign = 256;
+// Workspace header of a layer call: flag word at 0, router ticket at 64, down
+// tile-completion counters at 1024 (zeroed by moe_workspace_init).
+static constexpr size_t kHeaderBytes = 4096;
 static size_t up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 
 static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -64,7 +80,7 @@ bool plan_layer(int64_t T, int64_t H, int64_t I, const moe_router_cfg *cfg, int3
     const size_t E = static_cast<size_t>(p->E);
     const size_t Pall = P + static_cast<size_t>(T);
     size_t o = 0;
-    p->off_flags = o;   o = up(o + 256);
+    p->off_flags = o;   o = up(o + kHeaderBytes);
     p->off_part = o;    o = up(o + route_part_bytes(T, H, p->E));
     p->off_idx = o;     o = up(o + P * 4);
     p->off_w = o;       o = up(o + P * 4);
@@ -80,6 +96,20 @@ bool plan_layer(int64_t T, int64_t H, int64_t I, const moe_router_cfg *cfg, int3
     p->off_yp = o;      o = up(o + Pall * static_cast<size_t>(H) * 4);
     p->total = o;
     return true;
+}
+
+}  // namespace moe
+
+namespace moe {
+
+// Per-stage timing events.  Inside a stream capture they must be recorded as
+// external event nodes, or the graph keeps them as internal dependencies only.
+void record_stage_event(cudaEvent_t ev, cudaStream_t s) {
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(s, &cs) == cudaSuccess && cs == cudaStreamCaptureStatusActive)
+        cudaEventRecordWithFlags(ev, s, cudaEventRecordExternal);
+    else
+        cudaEventRecord(ev, s);
 }
 
 }  // namespace moe
@@ -106,7 +136,8 @@ int32_t moe_abi_version(void) { return 1; }
 
 moe_status moe_workspace_init(void *ws, size_t ws_bytes, cudaStream_t stream) {
     if (!ws || ws_bytes < 256) return MOE_ERR_WORKSPACE;
-    return CUDA_OK(cudaMemsetAsync(ws, 0, 256, stream)) ? MOE_OK : MOE_ERR_CUDA;
+    const size_t n = ws_bytes < kHeaderBytes ? ws_bytes : kHeaderBytes;
+    return CUDA_OK(cudaMemsetAsync(ws, 0, n, stream)) ? MOE_OK : MOE_ERR_CUDA;
 }
 
 moe_status moe_workspace_status(const void *ws, cudaStream_t stream, uint32_t *flags_out) {
@@ -192,7 +223,7 @@ size_t moe_layer_workspace_bytes(int64_t T, int64_t H, int64_t I, const moe_rout
 }
 
 static void rec(cudaEvent_t *ev, int i, cudaStream_t s) {
-    if (ev && ev[i]) cudaEventRecord(ev[i], s);
+    if (ev && ev[i]) record_stage_event(ev[i], s);
 }
 
 moe_status moe_layer_forward_ex(const uint16_t *x, int64_t T, int64_t H, int64_t I,
@@ -228,10 +259,31 @@ moe_status moe_layer_forward_ex(const uint16_t *x, int64_t T, int64_t H, int64_t
     float *h = reinterpret_cast<float *>(base + p.off_h);
     float *yp = reinterpret_cast<float *>(base + p.off_yp);
     moe_status st;
+    unsigned *counter = reinterpret_cast<unsigned *>(base + p.off_flags + 64);
+    int32_t *tile_cnt = reinterpret_cast<int32_t *>(base + p.off_flags + 1024);
+    float *logits = reinterpret_cast<float *>(base + p.off_part);
+
+    if (p.path == MOE_PATH_GEMV && route_fused_ok(T, H) && decode_ok(T, H, I, p.k, weight_bits)) {
+        // decode-size batch: fused router + bucketing, then the two GEMV kernels
+        rec(events, 0, stream);
+        st = launch_route_fused(x, T, H, gate, bias, cfg, idx, w, logits, counter, counts, offsets,
+                                list, tok, pos, unique, nunique, flags, tile_cnt,
+                                static_cast<int32_t>(H / 64), stream);
+        if (st != MOE_OK) return st;
+        rec(events, 1, stream);
+        rec(events, 2, stream);
+        st = run_decode_layer(x, T, H, I, p.k, weight_bits, experts, shared, unique, nunique,
+                              offsets, tok, pos, idx, w, h, yp, tile_cnt, y, accumulate, flags,
+                              stream, events ? events[3] : nullptr);
+        if (st != MOE_OK) return st;
+        rec(events, 4, stream);
+        rec(events, 5, stream);
+        return MOE_OK;
+    }
 
     rec(events, 0, stream);
     st = launch_route(x, T, H, gate, bias, cfg, idx, w, nullptr,
-                      reinterpret_cast<double *>(base + p.off_part), stream);
+                      reinterpret_cast<double *>(logits), stream);
     if (st != MOE_OK) return st;
     rec(events, 1, stream);
     st = launch_bucket(idx, T, p.k, p.E, counts, offsets, list, tok, pos, unique, nunique, flags, 0,

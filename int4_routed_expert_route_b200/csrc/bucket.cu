@@ -13,43 +13,6 @@ namespace moe {
 
 constexpr int BK_THREADS = 1024;
 
-__device__ __forceinline__ unsigned lanemask_lt() {
-    unsigned m;
-    asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
-    return m;
-}
-
-// Exclusive scan of one int per thread across the block; returns the prefix
-// and writes the block total to *total (all threads).
-__device__ int block_exclusive_scan(int v, int *warp_tot, int *total) {
-    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-    int inc = v;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const int n = __shfl_up_sync(0xffffffffu, inc, o);
-        if (lane >= o) inc += n;
-    }
-    if (lane == 31) warp_tot[wid] = inc;
-    __syncthreads();
-    if (wid == 0) {
-        const int nw = blockDim.x >> 5;
-        int t = lane < nw ? warp_tot[lane] : 0;
-        int ti = t;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int n = __shfl_up_sync(0xffffffffu, ti, o);
-            if (lane >= o) ti += n;
-        }
-        if (lane < nw) warp_tot[lane] = ti - t;  // exclusive warp offsets
-        if (lane == 31) warp_tot[32] = ti;
-    }
-    __syncthreads();
-    const int ex = warp_tot[wid] + inc - v;
-    *total = warp_tot[32];
-    __syncthreads();
-    return ex;
-}
-
 struct BucketArgs {
     const int32_t *idx;
     int64_t P;  // T * k

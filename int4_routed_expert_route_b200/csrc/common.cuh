@@ -46,6 +46,43 @@ __device__ __forceinline__ float warp_max(float v) {
     return v;
 }
 
+__device__ __forceinline__ unsigned lanemask_lt() {
+    unsigned m;
+    asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+    return m;
+}
+
+// Exclusive scan of one int per thread across the block; returns the prefix
+// and writes the block total to *total (all threads).
+__device__ __forceinline__ int block_exclusive_scan(int v, int *warp_tot, int *total) {
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    int inc = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int n = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc += n;
+    }
+    if (lane == 31) warp_tot[wid] = inc;
+    __syncthreads();
+    if (wid == 0) {
+        const int nw = blockDim.x >> 5;
+        int t = lane < nw ? warp_tot[lane] : 0;
+        int ti = t;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int n = __shfl_up_sync(0xffffffffu, ti, o);
+            if (lane >= o) ti += n;
+        }
+        if (lane < nw) warp_tot[lane] = ti - t;  // exclusive warp offsets
+        if (lane == 31) warp_tot[32] = ti;
+    }
+    __syncthreads();
+    const int ex = warp_tot[wid] + inc - v;
+    *total = warp_tot[32];
+    __syncthreads();
+    return ex;
+}
+
 // Packed pair of fp32 values in one 64-bit register (the sm_100 f32x2 datapath).
 struct f2 {
     unsigned long long v;
@@ -53,11 +90,29 @@ struct f2 {
 
 __device__ __forceinline__ f2 f2_make(float lo, float hi) {
     f2 r;
-    r.v = (static_cast<unsigned long long>(__float_as_uint(hi)) << 32) | __float_as_uint(lo);
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r.v) : "f"(lo), "f"(hi));
     return r;
 }
-__device__ __forceinline__ float f2_lo(f2 a) { return __uint_as_float(static_cast<uint32_t>(a.v)); }
-__device__ __forceinline__ float f2_hi(f2 a) { return __uint_as_float(static_cast<uint32_t>(a.v >> 32)); }
+__device__ __forceinline__ f2 f2_make_bits(uint32_t lo, uint32_t hi) {
+    f2 r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r.v) : "r"(lo), "r"(hi));
+    return r;
+}
+__device__ __forceinline__ float f2_lo(f2 a) {
+    float lo, hi;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(a.v));
+    return lo;
+}
+__device__ __forceinline__ float f2_hi(f2 a) {
+    float lo, hi;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(a.v));
+    return hi;
+}
+__device__ __forceinline__ float f2_sum(f2 a) {
+    float lo, hi;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(a.v));
+    return lo + hi;
+}
 
 // acc += a * b  (two lanes, round-to-nearest, no contraction surprises)
 __device__ __forceinline__ void f2_fma(f2 &acc, f2 a, f2 b) {

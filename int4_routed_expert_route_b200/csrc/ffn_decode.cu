@@ -1,0 +1,584 @@
+// ffn_decode.cu -- expert FFN for decode-size batches (T <= 8) on CUDA cores.
+//
+// Bandwidth design for HBM-bound int4 GEMV ("Show HN: running GLM 5.2 on a slow
+// computer", implemented features: dequant-on-use, batch-union MoE; here the
+// experts are resident in HBM instead of being streamed from disk):
+//  - Gate/up: the rows of all unique experts of the batch (shared expert first)
+//    form one row space; each block takes an equal contiguous range of it, so
+//    every SM streams the same number of bytes.  Warp (kw, rg) owns the 16-byte
+//    chunks [32kw, 32kw+32) of the rows rg, rg+RG, ... of the range; its slice of
+//    the activations stays in registers.  Each lane keeps two sets of U rows of
+//    128-bit streaming loads in flight (register double buffering).
+//  - Partial dot products are reduced across the warp with a reduce-scatter
+//    butterfly (V values in V-1 + log2(32/V) shuffles instead of 5V) and across
+//    the K-slice warps once per run in shared memory, in a fixed order.
+//  - Down: each block owns a contiguous range of output rows of H and loops
+//    over every unique expert of the batch, so it can apply the routing weights
+//    and the shared expert itself and write y once: the weighted combine is
+//    fused and deterministic (no atomics, no extra launch).
+#include <cstring>
+
+#include "common.cuh"
+#include "dequant.cuh"
+
+namespace moe {
+
+void record_stage_event(cudaEvent_t ev, cudaStream_t s);
+
+struct DecodeArgs {
+    const uint16_t *x;  // [T, H] bf16
+    int64_t T, H, I;
+    int32_t k;
+    const moe_expert *experts;  // device [E]
+    const moe_expert *shared;   // device, nullable
+    const int32_t *unique, *n_unique, *offsets, *tok, *pos, *idx;
+    const float *w;   // [T, k] routing weights
+    float *h;         // [T*k + T, I] fp32
+    float *y;         // [T, H] fp32
+    float *yp;        // [T*k + T, H] fp32 per-pair down outputs
+    int32_t *tile_cnt;  // [H / 64] completion counters (zero between calls)
+    int32_t accumulate;
+    int32_t kw, rg;   // K-slice warps, row groups (blockDim = 32 * kw * rg)
+    int32_t rows_pb;  // down: max output rows per block (smem sizing)
+    uint32_t *flags;
+};
+
+struct DSeg {
+    const moe_expert *ex;
+    const int32_t *toks;  // nullable: identity
+    int64_t n_tok;
+    int64_t hrow;
+};
+
+__device__ __forceinline__ int64_t dec_nseg(const DecodeArgs &a) {
+    return static_cast<int64_t>(*a.n_unique) + (a.shared ? 1 : 0);
+}
+
+// Segment 0 is the shared expert when present, then the unique routed experts.
+__device__ __forceinline__ DSeg dec_seg(const DecodeArgs &a, int64_t s) {
+    DSeg g;
+    if (a.shared) {
+        if (s == 0) {
+            g.ex = a.shared;
+            g.toks = nullptr;
+            g.n_tok = a.T;
+            g.hrow = a.T * a.k;
+            return g;
+        }
+        s -= 1;
+    }
+    const int e = a.unique[s];
+    const int o0 = a.offsets[e], o1 = a.offsets[e + 1];
+    g.ex = a.experts + e;
+    g.toks = a.tok + o0;
+    g.n_tok = o1 - o0;
+    g.hrow = o0;
+    return g;
+}
+
+__device__ __forceinline__ bool dqmat_ok(const moe_qmat &m, int bits, int64_t rows, int64_t cols) {
+    return m.q != nullptr && m.scale != nullptr && m.bits == bits && m.rows == rows && m.cols == cols;
+}
+
+// Reduce-scatter across the warp: V values per lane in, lane keeps the full
+// sum of value index bfly_index<V>(lane) in v[0].
+template <int V, int OFF>
+struct Bfly {
+    static __device__ __forceinline__ void run(float *v, int lane) {
+        const bool upper = (lane & OFF) != 0;
+#pragma unroll
+        for (int i = 0; i < V / 2; i++) {
+            const float send = upper ? v[i] : v[i + V / 2];
+            const float keep = upper ? v[i + V / 2] : v[i];
+            v[i] = keep + __shfl_xor_sync(0xffffffffu, send, OFF);
+        }
+        Bfly<V / 2, OFF / 2>::run(v, lane);
+    }
+};
+template <int OFF>
+struct Bfly<1, OFF> {
+    static __device__ __forceinline__ void run(float *v, int lane) {
+        v[0] += __shfl_xor_sync(0xffffffffu, v[0], OFF);
+        Bfly<1, OFF / 2>::run(v, lane);
+    }
+};
+template <>
+struct Bfly<1, 0> {
+    static __device__ __forceinline__ void run(float *, int) {}
+};
+
+template <int V>
+__device__ __forceinline__ int bfly_index(int lane) {
+    int idx = 0, half = V / 2, off = 16;
+#pragma unroll
+    for (int l = 0; l < 5; l++) {
+        if (half >= 1) {
+            if (lane & off) idx += half;
+            half >>= 1;
+        }
+        off >>= 1;
+    }
+    return idx;
+}
+
+// Lanes that write the reduced value (one per value index).
+template <int V>
+__device__ __forceinline__ bool bfly_writer(int lane) {
+    return (lane & (32 / V - 1)) == 0;
+}
+
+// 2^-e as an exact fp32 constant (0 <= e <= 20).
+__device__ __forceinline__ float exp2_neg(int e) { return __uint_as_float(static_cast<uint32_t>(127 - e) << 23); }
+
+// Loads a lane's activation slice (bf16 or fp32 source) pre-scaled by 2^-e.
+// f2 index w*PW + p = (column w*CPW + 2p, column w*CPW + 2p + 1), each
+// scaled by 2^-e of its code position.
+template <int BITS, typename Src>
+__device__ __forceinline__ float act_at(const Src *src, int col);
+template <>
+__device__ __forceinline__ float act_at<4, uint16_t>(const uint16_t *src, int col) { return bf16_bits_to_float(src[col]); }
+template <>
+__device__ __forceinline__ float act_at<8, uint16_t>(const uint16_t *src, int col) { return bf16_bits_to_float(src[col]); }
+template <>
+__device__ __forceinline__ float act_at<2, uint16_t>(const uint16_t *src, int col) { return bf16_bits_to_float(src[col]); }
+template <>
+__device__ __forceinline__ float act_at<4, float>(const float *src, int col) { return src[col]; }
+template <>
+__device__ __forceinline__ float act_at<8, float>(const float *src, int col) { return src[col]; }
+template <>
+__device__ __forceinline__ float act_at<2, float>(const float *src, int col) { return src[col]; }
+
+template <int BITS, typename Src>
+__device__ __forceinline__ void load_act(const Src *src, bool have, f2 *out) {
+    using D = Dec<BITS>;
+    constexpr int CW = Chunk<BITS>::W, PW = D::CPW / 2;
+    {
+#pragma unroll
+        for (int w = 0; w < CW; w++)
+#pragma unroll
+            for (int p = 0; p < PW; p++) {
+                float v0 = 0.f, v1 = 0.f;
+                if (have) {
+                    v0 = act_at<BITS, Src>(src, w * D::CPW + 2 * p) * exp2_neg(D::exp_of(2 * p));
+                    v1 = act_at<BITS, Src>(src, w * D::CPW + 2 * p + 1) * exp2_neg(D::exp_of(2 * p + 1));
+                }
+                out[w * PW + p] = f2_make(v0, v1);
+            }
+    }
+}
+
+// acc += decoded(chunk) . act  for one lane chunk.
+template <int BITS>
+__device__ __forceinline__ void chunk_fma(const uint32_t *wd, const f2 *act, f2 &acc) {
+    using D = Dec<BITS>;
+    constexpr int CW = Chunk<BITS>::W, PW = D::CPW / 2;
+    if constexpr (BITS == 4) {
+        const typename Dec<4>::Consts k = Dec<4>::consts();
+#pragma unroll
+        for (int w = 0; w < CW; w++) Dec<4>::dot(wd[w], act + w * PW, acc, k);
+    } else {
+#pragma unroll
+        for (int w = 0; w < CW; w++) {
+            f2 q[PW];
+            D::decode(wd[w], q);
+#pragma unroll
+            for (int p = 0; p < PW; p++) f2_fma(acc, q[p], act[w * PW + p]);
+        }
+    }
+}
+
+// Per-lane asynchronous copy ring.  Every lane prefetches exactly the chunks it
+// will consume into its own shared-memory slots (cp.async), S-1 steps ahead, and
+// waits only for its own copy groups: no barrier is needed, and the prefetch
+// depth no longer costs registers.
+template <int CH>
+__device__ __forceinline__ void cp_async_chunk(void *smem_dst, const void *gsrc) {
+    const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(smem_dst));
+    if constexpr (CH == 16)
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(gsrc) : "memory");
+    else
+        asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(d), "l"(gsrc) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+template <int BITS>
+__device__ __forceinline__ void lds_chunk(const uint8_t *p, uint32_t w[Chunk<BITS>::W]) {
+    if constexpr (Chunk<BITS>::W == 4) {
+        const uint4 v = *reinterpret_cast<const uint4 *>(p);
+        w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
+    } else {
+        const uint2 v = *reinterpret_cast<const uint2 *>(p);
+        w[0] = v.x; w[1] = v.y;
+    }
+}
+
+constexpr int DEC_RMAX = 128;  // rows per run (shared-memory partials)
+constexpr int GU_S = 4;        // gate/up copy-ring stages
+constexpr int DN_S = 8;        // down copy-ring stages
+constexpr int DN_RMAX = 512;   // rows per down run
+
+// ---------------------------------------------------------------------------
+// Gate/up + SwiGLU
+// ---------------------------------------------------------------------------
+template <int BITS, int TG, int U>
+__global__ void __launch_bounds__(384, 1) gateup_decode(DecodeArgs a) {
+    using D = Dec<BITS>;
+    constexpr int CW = Chunk<BITS>::W;
+    constexpr int NP = CW * (D::CPW / 2);
+    constexpr int V = U * 2 * TG;
+    extern __shared__ __align__(16) uint8_t dsm_gu[];
+    float *red = reinterpret_cast<float *>(dsm_gu);  // [DEC_RMAX][2][TG][KW]
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    uint8_t *ring_base = dsm_gu + static_cast<size_t>(DEC_RMAX) * 2 * TG * a.kw * sizeof(float);
+    const int KW = a.kw, RG = a.rg;
+    const int kw = warp % KW, rg = warp / KW;
+    const int64_t H = a.H, I = a.I;
+    const int64_t rb = H * BITS / 8;
+    const int64_t chunk = static_cast<int64_t>(kw) * 32 + lane;
+    const bool active = chunk * D::CH < rb;
+    const int64_t col0 = chunk * D::NC;
+    const int64_t R = dec_nseg(a) * I;
+    const int64_t r0 = R * blockIdx.x / gridDim.x, r1 = R * (blockIdx.x + 1) / gridDim.x;
+
+    f2 xs[TG][NP];
+    int64_t xs_seg = -1;
+    for (int64_t r = r0; r < r1;) {
+        const int64_t s = r / I;
+        const int64_t run_end = min(r1, (s + 1) * I);
+        const int64_t i_begin = r - s * I;
+        const DSeg g = dec_seg(a, s);
+        const moe_qmat mg = g.ex->gate, mu = g.ex->up;
+        const bool ok = dqmat_ok(mg, BITS, I, H) && dqmat_ok(mu, BITS, I, H);
+        if (!ok && threadIdx.x == 0) raise_flag(a.flags, MOE_FLAG_BAD_EXPERT_SHAPE);
+        for (int64_t sub = 0; ok && sub < run_end - r; sub += DEC_RMAX) {
+            const int m = static_cast<int>(run_end - r - sub < DEC_RMAX ? run_end - r - sub : DEC_RMAX);
+            const int64_t ib = i_begin + sub;  // first row (within the expert) of this sub-run
+            for (int64_t t0 = 0; t0 < g.n_tok; t0 += TG) {
+                if (xs_seg != s || g.n_tok > TG) {
+#pragma unroll
+                    for (int t = 0; t < TG; t++) {
+                        const bool have = active && t0 + t < g.n_tok;
+                        const int64_t tok = have ? (g.toks ? g.toks[t0 + t] : t0 + t) : 0;
+                        load_act<BITS, uint16_t>(a.x + tok * H + col0, have, xs[t]);
+                    }
+                    xs_seg = s;
+                }
+                const int nmy = rg < m ? (m - rg + RG - 1) / RG : 0;
+                const int nsteps = (nmy + U - 1) / U;
+                uint8_t *ring = ring_base + static_cast<size_t>(warp) * (GU_S * U * 2 * 32 * D::CH);
+                auto issue = [&](int step) {
+                    if (step < nsteps) {
+                        uint8_t *st = ring + static_cast<size_t>(step % GU_S) * (U * 2 * 32 * D::CH);
+#pragma unroll
+                        for (int u = 0; u < U; u++) {
+                            const int lr = rg + RG * (step * U + u);
+                            if (active && lr < m) {
+                                const int64_t row = ib + lr;
+                                cp_async_chunk<D::CH>(st + ((u * 2 + 0) * 32 + lane) * D::CH, mg.q + row * rb + chunk * D::CH);
+                                cp_async_chunk<D::CH>(st + ((u * 2 + 1) * 32 + lane) * D::CH, mu.q + row * rb + chunk * D::CH);
+                            }
+                        }
+                    }
+                    cp_async_commit();
+                };
+#pragma unroll
+                for (int st = 0; st < GU_S - 1; st++) issue(st);
+                for (int st = 0; st < nsteps; st++) {
+                    issue(st + GU_S - 1);
+                    cp_async_wait<GU_S - 1>();
+                    const uint8_t *sl = ring + static_cast<size_t>(st % GU_S) * (U * 2 * 32 * D::CH);
+                    uint32_t wr[U][2][CW];
+#pragma unroll
+                    for (int u = 0; u < U; u++)
+#pragma unroll
+                        for (int mm = 0; mm < 2; mm++) lds_chunk<BITS>(sl + ((u * 2 + mm) * 32 + lane) * D::CH, wr[u][mm]);
+                    float v[V];
+#pragma unroll
+                    for (int u = 0; u < U; u++)
+#pragma unroll
+                        for (int mm = 0; mm < 2; mm++)
+#pragma unroll
+                            for (int t = 0; t < TG; t++) {
+                                f2 acc;
+                                acc.v = 0ull;
+                                if (active) chunk_fma<BITS>(wr[u][mm], xs[t], acc);
+                                v[(u * 2 + mm) * TG + t] = f2_sum(acc);
+                            }
+                    Bfly<V, 16>::run(v, lane);
+                    if (bfly_writer<V>(lane)) {
+                        const int idx = bfly_index<V>(lane);
+                        const int u = idx / (2 * TG), mm = (idx / TG) % 2, t = idx % TG;
+                        const int lr = rg + RG * (st * U + u);
+                        if (lr < m) red[((lr * 2 + mm) * TG + t) * KW + kw] = v[0];
+                    }
+                }
+                cp_async_wait_all();
+                __syncthreads();
+                for (int q = threadIdx.x; q < m * TG; q += blockDim.x) {
+                    const int lr = q / TG, t = q % TG;
+                    if (t0 + t < g.n_tok) {
+                        float sg = 0.f, su = 0.f;
+                        for (int w = 0; w < KW; w++) {
+                            sg += red[((lr * 2 + 0) * TG + t) * KW + w];
+                            su += red[((lr * 2 + 1) * TG + t) * KW + w];
+                        }
+                        const int64_t row = ib + lr;
+                        const float gv = sg * mg.scale[row], uv = su * mu.scale[row];
+                        a.h[(g.hrow + t0 + t) * I + row] = silu(gv) * uv;
+                    }
+                }
+                __syncthreads();
+            }
+        }
+        r = run_end;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Down projection with the weighted combine fused.
+// Rows of all unique experts' down matrices form one row space split in equal
+// contiguous ranges (as for gate/up).  A block writes the unweighted per-pair
+// outputs yp[pair][j] = s_d[j] * (Q_d[j] . h_pair) of its rows, then counts the
+// rows it finished in every 64-row tile of H it touched; the block that
+// completes a tile (all segments done) combines it: y[t][j] = (y) +
+// sum_slot w * yp[pos(t,slot)][j] + yp[shared t][j], in slot order.
+// ---------------------------------------------------------------------------
+constexpr int DN_TILE = 64;
+constexpr int kMaxTiles = 768;  // counters live in the 4 KiB workspace header
+
+template <int BITS, int TG, int U>
+__global__ void __launch_bounds__(384, 1) down_decode(DecodeArgs a) {
+    using D = Dec<BITS>;
+    constexpr int CW = Chunk<BITS>::W;
+    constexpr int NP = CW * (D::CPW / 2);
+    constexpr int V = U * TG;
+    extern __shared__ __align__(16) uint8_t dsm_dn[];
+    float *red = reinterpret_cast<float *>(dsm_dn);  // [DN_RMAX][TG][KW]
+    uint8_t *ring_base = dsm_dn + static_cast<size_t>(DN_RMAX) * TG * a.kw * sizeof(float);
+    __shared__ int my_tiles[8];
+    __shared__ int n_my_tiles;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int KW = a.kw, RG = a.rg;
+    const int kw = warp % KW, rg = warp / KW;
+    const int64_t H = a.H, I = a.I, T = a.T;
+    const int64_t rb = I * BITS / 8;
+    const int64_t chunk = static_cast<int64_t>(kw) * 32 + lane;
+    const bool active = chunk * D::CH < rb;
+    const int64_t col0 = chunk * D::NC;
+    const int64_t nseg = dec_nseg(a);
+    const int64_t R = nseg * H;
+    const int64_t r0 = R * blockIdx.x / gridDim.x, r1 = R * (blockIdx.x + 1) / gridDim.x;
+
+    f2 hs[TG][NP];
+    for (int64_t r = r0; r < r1;) {
+        const int64_t s = r / H;
+        const int64_t run_end = min(r1, (s + 1) * H);
+        const int64_t j_begin = r - s * H;
+        const DSeg g = dec_seg(a, s);
+        const moe_qmat md = g.ex->down;
+        const bool ok = dqmat_ok(md, BITS, H, I);
+        if (!ok && threadIdx.x == 0) raise_flag(a.flags, MOE_FLAG_BAD_EXPERT_SHAPE);
+        for (int64_t sub = 0; sub < run_end - r; sub += DN_RMAX) {
+            const int m = static_cast<int>(run_end - r - sub < DN_RMAX ? run_end - r - sub : DN_RMAX);
+            const int64_t jb = j_begin + sub;
+            for (int64_t t0 = 0; ok && t0 < g.n_tok; t0 += TG) {
+#pragma unroll
+                for (int t = 0; t < TG; t++) {
+                    const bool have = active && t0 + t < g.n_tok;
+                    load_act<BITS, float>(a.h + (g.hrow + (have ? t0 + t : 0)) * I + col0, have, hs[t]);
+                }
+                const int nmy = rg < m ? (m - rg + RG - 1) / RG : 0;
+                const int nsteps = (nmy + U - 1) / U;
+                uint8_t *ring = ring_base + static_cast<size_t>(warp) * (DN_S * U * 32 * D::CH);
+                auto issue = [&](int step) {
+                    if (step < nsteps) {
+                        uint8_t *st = ring + static_cast<size_t>(step % DN_S) * (U * 32 * D::CH);
+#pragma unroll
+                        for (int u = 0; u < U; u++) {
+                            const int lr = rg + RG * (step * U + u);
+                            if (active && lr < m)
+                                cp_async_chunk<D::CH>(st + (u * 32 + lane) * D::CH, md.q + (jb + lr) * rb + chunk * D::CH);
+                        }
+                    }
+                    cp_async_commit();
+                };
+#pragma unroll
+                for (int st = 0; st < DN_S - 1; st++) issue(st);
+                for (int st = 0; st < nsteps; st++) {
+                    issue(st + DN_S - 1);
+                    cp_async_wait<DN_S - 1>();
+                    const uint8_t *sl = ring + static_cast<size_t>(st % DN_S) * (U * 32 * D::CH);
+                    uint32_t wr[U][CW];
+#pragma unroll
+                    for (int u = 0; u < U; u++) lds_chunk<BITS>(sl + (u * 32 + lane) * D::CH, wr[u]);
+                    float v[V];
+#pragma unroll
+                    for (int u = 0; u < U; u++)
+#pragma unroll
+                        for (int t = 0; t < TG; t++) {
+                            f2 acc;
+                            acc.v = 0ull;
+                            if (active) chunk_fma<BITS>(wr[u], hs[t], acc);
+                            v[u * TG + t] = f2_sum(acc);
+                        }
+                    Bfly<V, 16>::run(v, lane);
+                    if (bfly_writer<V>(lane)) {
+                        const int idx = bfly_index<V>(lane);
+                        const int u = idx / TG, t = idx % TG;
+                        const int lr = rg + RG * (st * U + u);
+                        if (lr < m) red[(lr * TG + t) * KW + kw] = v[0];
+                    }
+                }
+                cp_async_wait_all();
+                __syncthreads();
+                for (int q = threadIdx.x; q < m * TG; q += blockDim.x) {
+                    const int lr = q / TG, t = q % TG;
+                    if (t0 + t < g.n_tok) {
+                        float d = 0.f;
+                        for (int w = 0; w < KW; w++) d += red[(lr * TG + t) * KW + w];
+                        const int64_t j = jb + lr;
+                        a.yp[(g.hrow + t0 + t) * H + j] = d * md.scale[j];
+                    }
+                }
+                __syncthreads();
+            }
+            // completion accounting for the 64-row tiles this sub-run touched
+            __threadfence();
+            __syncthreads();
+            if (threadIdx.x == 0) {
+                n_my_tiles = 0;
+                const int64_t ja = jb, je = jb + m;
+                for (int64_t c = ja / DN_TILE; c * DN_TILE < je; c++) {
+                    const int64_t lo = c * DN_TILE > ja ? c * DN_TILE : ja;
+                    const int64_t hi = (c + 1) * DN_TILE < je ? (c + 1) * DN_TILE : je;
+                    const int add = static_cast<int>(hi - lo);
+                    const int need = static_cast<int>(nseg * DN_TILE);
+                    const int old = atomicAdd(a.tile_cnt + c, add);
+                    if (old + add == need) my_tiles[n_my_tiles++] = static_cast<int>(c);
+                }
+            }
+            __syncthreads();
+            const int nt = n_my_tiles;
+            if (nt > 0) __threadfence();
+            for (int i = 0; i < nt; i++) {
+                const int64_t c = my_tiles[i];
+                for (int q = threadIdx.x; q < DN_TILE * T; q += blockDim.x) {
+                    const int64_t t = q / DN_TILE;
+                    const int64_t j = c * DN_TILE + q % DN_TILE;
+                    float acc = a.accumulate ? a.y[t * H + j] : 0.0f;
+                    for (int sl = 0; sl < a.k; sl++) {
+                        const int p = a.pos[t * a.k + sl];
+                        if (p < 0) continue;
+                        acc += a.w[t * a.k + sl] * __ldcg(a.yp + static_cast<int64_t>(p) * H + j);
+                    }
+                    if (a.shared) acc += __ldcg(a.yp + (T * a.k + t) * H + j);
+                    a.y[t * H + j] = acc;
+                }
+                if (threadIdx.x == 0) a.tile_cnt[c] = 0;
+            }
+        }
+        r = run_end;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Host side
+// ---------------------------------------------------------------------------
+static int dec_sm_count() {
+    int dev = 0, n = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    return n;
+}
+
+static constexpr int DEC_U = 4;
+
+bool decode_ok(int64_t T, int64_t H, int64_t I, int32_t k, int32_t bits) {
+    (void)k;
+    if (T < 1 || T > 8 || H % 64 || I % 64 || H / DN_TILE > kMaxTiles) return false;
+    const int ch = bits == 2 ? 8 : 16;
+    const int64_t kw_gu = (H * bits / 8 / ch + 31) / 32, kw_dn = (I * bits / 8 / ch + 31) / 32;
+    return kw_gu <= 12 && kw_dn <= 12;
+}
+
+template <int BITS, int TG>
+static moe_status launch_decode_bits(DecodeArgs a, cudaStream_t stream, cudaEvent_t ev_down) {
+    using D = Dec<BITS>;
+    const int sms = dec_sm_count();
+    const int64_t rb_gu = a.H * BITS / 8, rb_dn = a.I * BITS / 8;
+    const int kw_gu = static_cast<int>((rb_gu / D::CH + 31) / 32);
+    const int kw_dn = static_cast<int>((rb_dn / D::CH + 31) / 32);
+    {
+        DecodeArgs g = a;
+        g.kw = kw_gu;
+        g.rg = 12 / kw_gu > 0 ? 12 / kw_gu : 1;
+        const int threads = 32 * g.kw * g.rg;
+        const size_t smem = static_cast<size_t>(DEC_RMAX) * 2 * TG * g.kw * sizeof(float) +
+                            static_cast<size_t>(threads / 32) * GU_S * DEC_U * 2 * 32 * D::CH;
+        auto kern = gateup_decode<BITS, TG, DEC_U>;
+        if (smem > 48 * 1024 &&
+            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        kern<<<sms, threads, smem, stream>>>(g);
+        if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
+    }
+    if (ev_down) record_stage_event(ev_down, stream);
+    {
+        DecodeArgs d = a;
+        d.kw = kw_dn;
+        d.rg = 12 / kw_dn > 0 ? 12 / kw_dn : 1;
+        const int threads = 32 * d.kw * d.rg;
+        const size_t smem = static_cast<size_t>(DN_RMAX) * TG * d.kw * sizeof(float) +
+                            static_cast<size_t>(threads / 32) * DN_S * DEC_U * 32 * D::CH;
+        auto kern = down_decode<BITS, TG, DEC_U>;
+        if (smem > 48 * 1024 &&
+            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        kern<<<sms, threads, smem, stream>>>(d);
+        if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
+    }
+    return MOE_OK;
+}
+
+moe_status run_decode_layer(const uint16_t *x, int64_t T, int64_t H, int64_t I, int32_t k,
+                            int32_t bits, const moe_expert *experts, const moe_expert *shared,
+                            const int32_t *unique, const int32_t *n_unique, const int32_t *offsets,
+                            const int32_t *tok, const int32_t *pos, const int32_t *idx,
+                            const float *w, float *h, float *yp, int32_t *tile_cnt, float *y,
+                            int32_t accumulate, uint32_t *flags, cudaStream_t stream,
+                            cudaEvent_t ev_down) {
+    DecodeArgs a;
+    std::memset(&a, 0, sizeof(a));
+    a.x = x;
+    a.T = T;
+    a.H = H;
+    a.I = I;
+    a.k = k;
+    a.experts = experts;
+    a.shared = shared;
+    a.unique = unique;
+    a.n_unique = n_unique;
+    a.offsets = offsets;
+    a.tok = tok;
+    a.pos = pos;
+    a.idx = idx;
+    a.w = w;
+    a.h = h;
+    a.y = y;
+    a.yp = yp;
+    a.tile_cnt = tile_cnt;
+    a.accumulate = accumulate;
+    a.flags = flags;
+    const bool tg1 = T == 1;
+    switch (bits) {
+    case 4: return tg1 ? launch_decode_bits<4, 1>(a, stream, ev_down) : launch_decode_bits<4, 2>(a, stream, ev_down);
+    case 8: return tg1 ? launch_decode_bits<8, 1>(a, stream, ev_down) : launch_decode_bits<8, 2>(a, stream, ev_down);
+    case 2: return launch_decode_bits<2, 1>(a, stream, ev_down);
+    default: return MOE_ERR_INVALID_ARG;
+    }
+}
+
+}  // namespace moe

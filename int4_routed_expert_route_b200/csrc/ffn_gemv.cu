@@ -24,98 +24,11 @@
 #include <cstring>
 
 #include "common.cuh"
+#include "dequant.cuh"
 
 namespace moe {
 
-// ---------------------------------------------------------------------------
-// Per-bit-width decode tables.
-// ---------------------------------------------------------------------------
-template <int BITS>
-struct Dec;
-
-// int4: 8 codes per word; nibbles 0..4 in place, 5..7 after >> 12.
-template <>
-struct Dec<4> {
-    static constexpr int CH = 16;                  // bytes per lane chunk
-    static constexpr int NC = CH * 8 / 4;          // codes per lane chunk (32)
-    static constexpr int CPW = 8;                  // codes per 32-bit word
-    __device__ static __forceinline__ int exp_of(int p) {
-        return (p < 5) ? 4 * p : 4 * (p - 3);      // 0 4 8 12 16 8 12 16
-    }
-    __device__ static __forceinline__ float bias_of() { return 8.0f; }
-    // q * 2^e for the 8 codes of word v, as 4 f32x2 pairs
-    __device__ static __forceinline__ void decode(uint32_t v, f2 out[4]) {
-        const uint32_t v2 = v >> 12;
-        const uint32_t M = 0x4B000000u;
-        const float c0 = 8388608.0f + 8.0f, c4 = 8388608.0f + 128.0f, c8 = 8388608.0f + 2048.0f,
-                    c12 = 8388608.0f + 32768.0f, c16 = 8388608.0f + 524288.0f;
-        out[0] = f2_sub(f2_make(__uint_as_float(M | (v & 0xFu)), __uint_as_float(M | (v & 0xF0u))), f2_make(c0, c4));
-        out[1] = f2_sub(f2_make(__uint_as_float(M | (v & 0xF00u)), __uint_as_float(M | (v & 0xF000u))), f2_make(c8, c12));
-        out[2] = f2_sub(f2_make(__uint_as_float(M | (v & 0xF0000u)), __uint_as_float(M | (v2 & 0xF00u))), f2_make(c16, c8));
-        out[3] = f2_sub(f2_make(__uint_as_float(M | (v2 & 0xF000u)), __uint_as_float(M | (v2 & 0xF0000u))), f2_make(c12, c16));
-    }
-};
-
-// int8: 4 two's-complement bytes per word; bias 128 after xor 0x80.
-template <>
-struct Dec<8> {
-    static constexpr int CH = 16;
-    static constexpr int NC = CH;                  // 16
-    static constexpr int CPW = 4;
-    __device__ static __forceinline__ int exp_of(int p) { return (p & 1) ? 8 : 0; }
-    __device__ static __forceinline__ void decode(uint32_t v, f2 out[2]) {
-        const uint32_t u = v ^ 0x80808080u;
-        const uint32_t u2 = u >> 16;
-        const uint32_t M = 0x4B000000u;
-        const float c0 = 8388608.0f + 128.0f, c8 = 8388608.0f + 32768.0f;
-        out[0] = f2_sub(f2_make(__uint_as_float(M | (u & 0xFFu)), __uint_as_float(M | (u & 0xFF00u))), f2_make(c0, c8));
-        out[1] = f2_sub(f2_make(__uint_as_float(M | (u2 & 0xFFu)), __uint_as_float(M | (u2 & 0xFF00u))), f2_make(c0, c8));
-    }
-};
-
-// int2: 16 crumbs per word; crumbs 0..9 in place, 10..15 after >> 20.
-template <>
-struct Dec<2> {
-    static constexpr int CH = 8;
-    static constexpr int NC = CH * 8 / 2;          // 32
-    static constexpr int CPW = 16;
-    __device__ static __forceinline__ int exp_of(int p) { return (p < 10) ? 2 * p : 2 * (p - 10); }
-    __device__ static __forceinline__ void decode(uint32_t v, f2 out[8]) {
-        const uint32_t v2 = v >> 20;
-        const uint32_t M = 0x4B000000u;
-#pragma unroll
-        for (int i = 0; i < 8; i++) {
-            const int p0 = 2 * i, p1 = 2 * i + 1;
-            const uint32_t w0 = (p0 < 10) ? (v & (3u << (2 * p0))) : (v2 & (3u << (2 * (p0 - 10))));
-            const uint32_t w1 = (p1 < 10) ? (v & (3u << (2 * p1))) : (v2 & (3u << (2 * (p1 - 10))));
-            const int e0 = (p0 < 10) ? 2 * p0 : 2 * (p0 - 10);
-            const int e1 = (p1 < 10) ? 2 * p1 : 2 * (p1 - 10);
-            out[i] = f2_sub(f2_make(__uint_as_float(M | w0), __uint_as_float(M | w1)),
-                            f2_make(8388608.0f + 2.0f * static_cast<float>(1u << e0),
-                                    8388608.0f + 2.0f * static_cast<float>(1u << e1)));
-        }
-    }
-};
-
-template <int BITS>
-struct Chunk;
-template <>
-struct Chunk<4> { using T = uint4; static constexpr int W = 4; };
-template <>
-struct Chunk<8> { using T = uint4; static constexpr int W = 4; };
-template <>
-struct Chunk<2> { using T = uint2; static constexpr int W = 2; };
-
-template <int BITS>
-__device__ __forceinline__ void load_chunk(const uint8_t *p, uint32_t w[Chunk<BITS>::W]) {
-    if constexpr (Chunk<BITS>::W == 4) {
-        const uint4 v = ldg_stream(p);
-        w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
-    } else {
-        const uint2 v = ldg_stream8(p);
-        w[0] = v.x; w[1] = v.y;
-    }
-}
+void record_stage_event(cudaEvent_t ev, cudaStream_t s);
 
 // ---------------------------------------------------------------------------
 // Arguments and segment resolution.
@@ -559,7 +472,7 @@ moe_status run_gemv_layer(const uint16_t *x, int64_t T, int64_t H, int64_t I, in
     a.flags = flags;
     moe_status st = launch_gemv(a, max_segments, max_tok, stream, true, false);
     if (st != MOE_OK) return st;
-    if (ev_down) cudaEventRecord(ev_down, stream);
+    if (ev_down) record_stage_event(ev_down, stream);
     return launch_gemv(a, max_segments, max_tok, stream, false, true);
 }
 

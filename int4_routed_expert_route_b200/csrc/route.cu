@@ -17,52 +17,63 @@
 namespace moe {
 
 // ---------------------------------------------------------------------------
-// Logits for small batches: one warp per (expert, K-slice); the warp keeps its
-// slice of the gate row in registers and loops over the tokens.
-// part[ks][t][e] = sum over the slice of G[e,j] * x[t,j], fp64.
+// Logits for small batches: one block per expert, its 8 warps split the hidden
+// dimension; exact bf16*fp32 products are accumulated in fp64, the 8 slice
+// sums are added in a fixed order and the total is rounded once to fp32.
+// logits[t][e] (fp32).  T <= 64.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) route_logits_small(const uint16_t *__restrict__ x,
-                                                          int64_t T, int64_t H,
-                                                          const float *__restrict__ G, int E,
-                                                          int KS, double *__restrict__ part) {
-    const int lane = threadIdx.x & 31;
-    const int e = blockIdx.x * 8 + (threadIdx.x >> 5);
-    const int ks = blockIdx.y;
-    if (e >= E) return;
-    const int64_t L = H / KS;
-    const int64_t k0 = static_cast<int64_t>(ks) * L;
-    constexpr int MAXV = 4;  // up to 4 float4 per lane held in registers (L <= 512)
-    float4 g[MAXV];
-    int nv = 0;
+constexpr int RL_WARPS = 8;
+constexpr int RL_MAXT = 64;
+
+__device__ __forceinline__ double dot4(float4 g, uint2 xv, double acc) {
+    acc = fma(static_cast<double>(g.x), static_cast<double>(bf16_bits_to_float(xv.x & 0xffffu)), acc);
+    acc = fma(static_cast<double>(g.y), static_cast<double>(bf16_bits_to_float(xv.x >> 16)), acc);
+    acc = fma(static_cast<double>(g.z), static_cast<double>(bf16_bits_to_float(xv.y & 0xffffu)), acc);
+    acc = fma(static_cast<double>(g.w), static_cast<double>(bf16_bits_to_float(xv.y >> 16)), acc);
+    return acc;
+}
+
+// Block-level body: computes logits[t][e] for t < T of expert e = blockIdx.x.
+__device__ void logits_one_expert(const uint16_t *__restrict__ x, int64_t T, int64_t H,
+                                  const float *__restrict__ G, int E, float *__restrict__ logits,
+                                  double *red /* [RL_WARPS][RL_MAXT] smem */) {
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    const int e = blockIdx.x;
+    const int64_t L = H / RL_WARPS;  // H % 512 == 0 -> L % 64 == 0
+    const int64_t k0 = static_cast<int64_t>(wid) * L;
+    const float *gr = G + static_cast<int64_t>(e) * H + k0;
+    for (int64_t t0 = 0; t0 < T; t0 += 4) {
+        double acc[4] = {0.0, 0.0, 0.0, 0.0};
+        for (int64_t j = 4 * lane; j < L; j += 128) {
+            const float4 g = *reinterpret_cast<const float4 *>(gr + j);
 #pragma unroll
-    for (int v = 0; v < MAXV; v++) {
-        const int64_t j = 4 * lane + 128 * v;
-        if (j < L) {
-            g[v] = *reinterpret_cast<const float4 *>(G + static_cast<int64_t>(e) * H + k0 + j);
-            nv = v + 1;
-        } else {
-            g[v] = make_float4(0.f, 0.f, 0.f, 0.f);
-        }
-    }
-    for (int64_t t = 0; t < T; t++) {
-        double acc = 0.0;
-        const uint16_t *xr = x + t * H + k0;
-#pragma unroll
-        for (int v = 0; v < MAXV; v++) {
-            if (v < nv) {
-                const int64_t j = 4 * lane + 128 * v;
-                if (j < L) {
-                    const uint2 xv = *reinterpret_cast<const uint2 *>(xr + j);
-                    acc = fma(static_cast<double>(g[v].x), static_cast<double>(bf16_bits_to_float(xv.x & 0xffffu)), acc);
-                    acc = fma(static_cast<double>(g[v].y), static_cast<double>(bf16_bits_to_float(xv.x >> 16)), acc);
-                    acc = fma(static_cast<double>(g[v].z), static_cast<double>(bf16_bits_to_float(xv.y & 0xffffu)), acc);
-                    acc = fma(static_cast<double>(g[v].w), static_cast<double>(bf16_bits_to_float(xv.y >> 16)), acc);
+            for (int u = 0; u < 4; u++) {
+                if (t0 + u < T) {
+                    const uint2 xv = *reinterpret_cast<const uint2 *>(x + (t0 + u) * H + k0 + j);
+                    acc[u] = dot4(g, xv, acc[u]);
                 }
             }
         }
-        acc = warp_sum(acc);
-        if (lane == 0) part[(static_cast<int64_t>(ks) * T + t) * E + e] = acc;
+#pragma unroll
+        for (int u = 0; u < 4; u++) {
+            const double v = warp_sum(acc[u]);
+            if (lane == 0 && t0 + u < T) red[wid * RL_MAXT + t0 + u] = v;
+        }
     }
+    __syncthreads();
+    for (int64_t t = threadIdx.x; t < T; t += blockDim.x) {
+        double v = 0.0;
+        for (int w = 0; w < RL_WARPS; w++) v += red[w * RL_MAXT + t];
+        logits[t * E + e] = static_cast<float>(v);
+    }
+}
+
+__global__ void __launch_bounds__(RL_WARPS * 32) route_logits_small(const uint16_t *__restrict__ x,
+                                                                    int64_t T, int64_t H,
+                                                                    const float *__restrict__ G,
+                                                                    int E, float *__restrict__ logits) {
+    __shared__ double red[RL_WARPS * RL_MAXT];
+    logits_one_expert(x, T, H, G, E, logits, red);
 }
 
 // ---------------------------------------------------------------------------
@@ -75,7 +86,7 @@ constexpr int RT_T = 64, RT_E = 64, RT_K = 32;
 __global__ void __launch_bounds__(256) route_logits_tiled(const uint16_t *__restrict__ x,
                                                           int64_t T, int64_t H,
                                                           const float *__restrict__ G, int E,
-                                                          double *__restrict__ part) {
+                                                          float *__restrict__ logits) {
     __shared__ float xs[RT_K][RT_T + 4];
     __shared__ float gs[RT_K][RT_E + 4];
     const int tid = threadIdx.x;
@@ -143,7 +154,7 @@ __global__ void __launch_bounds__(256) route_logits_tiled(const uint16_t *__rest
 #pragma unroll
         for (int j = 0; j < 4; j++) {
             const int e = e0 + tx * 4 + j;
-            if (e < E) part[t * E + e] = dacc[i][j];
+            if (e < E) logits[t * E + e] = static_cast<float>(dacc[i][j]);
         }
     }
 }
@@ -152,8 +163,7 @@ __global__ void __launch_bounds__(256) route_logits_tiled(const uint16_t *__rest
 // Selection: one warp per token.
 // ---------------------------------------------------------------------------
 struct SelArgs {
-    const double *part;
-    int KS;
+    const float *logits;  // [T][E] fp32
     int64_t T;
     const float *bias;
     int E, k, n_group, topk_group;
@@ -178,27 +188,16 @@ __device__ __forceinline__ void warp_argmax(float &v, int &i) {
 
 constexpr int SEL_WARPS = 4;
 
-__global__ void __launch_bounds__(SEL_WARPS * 32) route_select(SelArgs a) {
-    extern __shared__ float smem[];
-    const int lane = threadIdx.x & 31;
-    const int wid = threadIdx.x >> 5;
-    const int64_t t = static_cast<int64_t>(blockIdx.x) * SEL_WARPS + wid;
-    if (t >= a.T) return;
-    const int E = a.E;
-    float *s_sm = smem + wid * (2 * E + 64);
-    float *b_sm = s_sm + E;
-    float *g_sm = b_sm + E;          // group scores [<=32]
-    int *pick = reinterpret_cast<int *>(g_sm + 32);  // chosen experts [<=32]
+// Sigmoid score of one logit: evaluated in fp64, rounded to fp32.
+__device__ __forceinline__ float sigmoid_score(float logit) {
+    return static_cast<float>(1.0 / (1.0 + exp(-static_cast<double>(logit))));
+}
 
-    for (int e = lane; e < E; e += 32) {
-        double l = 0.0;
-        for (int ks = 0; ks < a.KS; ks++) l += a.part[(static_cast<int64_t>(ks) * a.T + t) * E + e];
-        const float logit = static_cast<float>(l);
-        const float s = static_cast<float>(1.0 / (1.0 + exp(-static_cast<double>(logit))));
-        s_sm[e] = s;
-        b_sm[e] = s + a.bias[e];
-    }
-    __syncwarp();
+// Selection of token t by one warp from its scores s_sm[E] and biased scores
+// b_sm[E] in shared memory (b_sm is consumed); pick is 32 ints of scratch.
+__device__ void select_core(const SelArgs &a, int64_t t, const float *s_sm, float *b_sm, int *pick) {
+    const int lane = threadIdx.x & 31;
+    const int E = a.E;
 
     const int ng = a.n_group, gsz = E / ng;
     float gscore = -INFINITY;
@@ -317,38 +316,167 @@ __global__ void __launch_bounds__(SEL_WARPS * 32) route_select(SelArgs a) {
     }
 }
 
-// K-splits for the small-batch logits: slices of at most 512 columns (the
-// registers a lane holds), a multiple of 4 columns each.  H % 64 == 0.
-int route_ks_for(int64_t T, int64_t H) {
-    if (T > 64) return 1;
-    for (int64_t ks = (H + 511) / 512; ks <= H / 4; ks++)
-        if (H % ks == 0 && (H / ks) % 4 == 0) return static_cast<int>(ks);
-    return static_cast<int>(H / 4);
-}
-
-size_t route_part_bytes(int64_t T, int64_t H, int E) {
-    return static_cast<size_t>(route_ks_for(T, H)) * static_cast<size_t>(T) * E * sizeof(double);
-}
-
-moe_status launch_route(const uint16_t *x, int64_t T, int64_t H, const float *gate,
-                        const float *bias, const moe_router_cfg *cfg, int32_t *idx_out,
-                        float *w_out, float *gap_out, double *part, cudaStream_t stream) {
-    if (T == 0) return MOE_OK;
-    const int E = cfg->n_experts;
-    const int KS = route_ks_for(T, H);
-    if (T <= 64) {
-        dim3 grid((E + 7) / 8, KS);
-        route_logits_small<<<grid, 256, 0, stream>>>(x, T, H, gate, E, KS, part);
-    } else {
-        dim3 grid(static_cast<unsigned>((T + RT_T - 1) / RT_T), (E + RT_E - 1) / RT_E);
-        route_logits_tiled<<<grid, 256, 0, stream>>>(x, T, H, gate, E, part);
+// Routes token t with one warp; wsm is this warp's shared scratch of
+// (2E + 64) floats.
+__device__ void select_token(const SelArgs &a, int64_t t, float *wsm) {
+    const int lane = threadIdx.x & 31;
+    const int E = a.E;
+    float *s_sm = wsm;
+    float *b_sm = s_sm + E;
+    int *pick = reinterpret_cast<int *>(b_sm + E + 32);
+    for (int e = lane; e < E; e += 32) {
+        const float sc = sigmoid_score(__ldcg(a.logits + t * E + e));
+        s_sm[e] = sc;
+        b_sm[e] = sc + a.bias[e];
     }
+    __syncwarp();
+    select_core(a, t, s_sm, b_sm, pick);
+}
+
+__global__ void __launch_bounds__(SEL_WARPS * 32) route_select(SelArgs a) {
+    extern __shared__ float smem[];
+    const int wid = threadIdx.x >> 5;
+    const int64_t t = static_cast<int64_t>(blockIdx.x) * SEL_WARPS + wid;
+    if (t >= a.T) return;
+    select_token(a, t, smem + wid * (2 * a.E + 64));
+}
+
+// ---------------------------------------------------------------------------
+// Decode-size batches (T <= 8): logits, selection and batch-union bucketing in
+// one launch.  Every block computes one expert's logits; the last block to
+// finish (ticket counter in the workspace header) routes the tokens with its 8
+// warps and then buckets the (token, slot) pairs with a stable counting sort.
+// The counter is reset by that block for the next call.
+// ---------------------------------------------------------------------------
+constexpr int FUSED_MAXT = 8;
+
+struct FusedRouteArgs {
+    const uint16_t *x;
+    int64_t H;
+    const float *G;
+    float *logits;
+    SelArgs sel;
+    unsigned *counter;
+    int32_t *counts, *offsets, *list, *tok, *pos, *unique, *n_unique;
+    uint32_t *flags;
+    int32_t *zero_cnt;  // counters of the following kernels, cleared here
+    int32_t n_zero;
+};
+
+// Stable counting sort of P <= 32 * 2048 pairs by one block (sm: E + 48 ints).
+__device__ void bucket_small(const int32_t *idx, int P, int k, int E, int32_t *counts,
+                             int32_t *offsets, int32_t *list, int32_t *tok, int32_t *pos,
+                             int32_t *unique, int32_t *n_unique, uint32_t *flags, int *sm) {
+    int *cur = sm;
+    int *wt = sm + E;
+    const int tid = threadIdx.x, lane = tid & 31;
+    for (int e = tid; e < E; e += blockDim.x) cur[e] = 0;
+    __syncthreads();
+    bool bad = false;
+    for (int p = tid; p < P; p += blockDim.x) {
+        const int e = __ldcg(idx + p);
+        if (e >= E) bad = true;
+        else if (e >= 0) atomicAdd(&cur[e], 1);
+    }
+    if (__syncthreads_or(bad) && tid == 0) raise_flag(flags, MOE_FLAG_BAD_EXPERT_INDEX);
+    const int per = (E + blockDim.x - 1) / blockDim.x;
+    const int e0 = tid * per, e1 = min(E, e0 + per);
+    int c = 0, nz = 0;
+    for (int e = e0; e < e1; e++) {
+        c += cur[e];
+        nz += cur[e] > 0;
+    }
+    int tot, nu;
+    const int off = block_exclusive_scan(c, wt, &tot);
+    const int uo = block_exclusive_scan(nz, wt, &nu);
+    int run = off, u = uo;
+    for (int e = e0; e < e1; e++) {
+        const int ce = cur[e];
+        counts[e] = ce;
+        offsets[e] = run;
+        if (ce > 0) unique[u++] = e;
+        cur[e] = run;
+        run += ce;
+    }
+    if (tid == 0) {
+        offsets[E] = tot;
+        *n_unique = nu;
+    }
+    __syncthreads();
+    if (tid < 32) {
+        for (int base = 0; base < P; base += 32) {
+            const int p = base + lane;
+            const int e = p < P ? __ldcg(idx + p) : -1;
+            const bool valid = e >= 0 && e < E;
+            const unsigned mask = __match_any_sync(0xffffffffu, valid ? e : -1);
+            const int rank = __popc(mask & lanemask_lt());
+            const bool leader = (__ffs(mask) - 1) == lane;
+            int q = -1;
+            if (valid) q = cur[e] + rank;
+            __syncwarp();
+            if (valid) {
+                list[q] = p;
+                tok[q] = p / k;
+                if (leader) cur[e] += __popc(mask);
+            }
+            if (p < P) pos[p] = q;
+            __syncwarp();
+        }
+    }
+}
+
+__global__ void __launch_bounds__(RL_WARPS * 32) route_fused_small(FusedRouteArgs a) {
+    extern __shared__ float dsm[];
+    __shared__ double red[RL_WARPS * RL_MAXT];
+    __shared__ unsigned ticket;
+    logits_one_expert(a.x, a.sel.T, a.H, a.G, a.sel.E, a.logits, red);
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) ticket = atomicAdd(a.counter, 1u);
+    __syncthreads();
+    if (ticket != gridDim.x - 1) return;
+    __threadfence();
+    const int wid = threadIdx.x >> 5;
+    const int E = a.sel.E;
+    const int64_t T = a.sel.T;
+    float *s_all = dsm;               // [T][E]
+    float *b_all = dsm + T * E;       // [T][E]
+    int *picks = reinterpret_cast<int *>(b_all + T * E);  // [8][32]
+    for (int64_t i = threadIdx.x; i < T * E; i += blockDim.x) {
+        const int e = static_cast<int>(i % E);
+        const float sc = sigmoid_score(__ldcg(a.logits + i));
+        s_all[i] = sc;
+        b_all[i] = sc + a.sel.bias[e];
+    }
+    __syncthreads();
+    for (int64_t t = wid; t < T; t += RL_WARPS)
+        select_core(a.sel, t, s_all + t * E, b_all + t * E, picks + wid * 32);
+    __syncthreads();
+    bucket_small(a.sel.idx_out, static_cast<int>(a.sel.T * a.sel.k), a.sel.k, E, a.counts, a.offsets,
+                 a.list, a.tok, a.pos, a.unique, a.n_unique, a.flags, reinterpret_cast<int *>(dsm));
+    for (int i = threadIdx.x; i < a.n_zero; i += blockDim.x) a.zero_cnt[i] = 0;
+    if (threadIdx.x == 0) *a.counter = 0u;
+}
+
+// Scratch of the router: fp32 logits [T][E].
+size_t route_part_bytes(int64_t T, int64_t H, int E) {
+    (void)H;
+    return static_cast<size_t>(T) * E * sizeof(float);
+}
+
+int route_ks_for(int64_t T, int64_t H) {
+    (void)T;
+    (void)H;
+    return 1;
+}
+
+static SelArgs sel_args(int64_t T, const float *bias, const moe_router_cfg *cfg, int32_t *idx_out,
+                        float *w_out, float *gap_out, const float *logits) {
     SelArgs a;
-    a.part = part;
-    a.KS = KS;
+    a.logits = logits;
     a.T = T;
     a.bias = bias;
-    a.E = E;
+    a.E = cfg->n_experts;
     a.k = cfg->top_k;
     a.n_group = cfg->n_group;
     a.topk_group = cfg->topk_group;
@@ -357,9 +485,64 @@ moe_status launch_route(const uint16_t *x, int64_t T, int64_t H, const float *ga
     a.idx_out = idx_out;
     a.w_out = w_out;
     a.gap_out = gap_out;
-    const size_t smem = SEL_WARPS * (2 * E + 64) * sizeof(float);
+    return a;
+}
+
+static size_t sel_smem(int E, int warps) { return static_cast<size_t>(warps) * (2 * E + 64) * sizeof(float); }
+
+moe_status launch_route(const uint16_t *x, int64_t T, int64_t H, const float *gate,
+                        const float *bias, const moe_router_cfg *cfg, int32_t *idx_out,
+                        float *w_out, float *gap_out, double *scratch, cudaStream_t stream) {
+    if (T == 0) return MOE_OK;
+    const int E = cfg->n_experts;
+    float *logits = reinterpret_cast<float *>(scratch);
+    if (T <= RL_MAXT && H % 32 == 0) {
+        route_logits_small<<<E, RL_WARPS * 32, 0, stream>>>(x, T, H, gate, E, logits);
+    } else {
+        dim3 grid(static_cast<unsigned>((T + RT_T - 1) / RT_T), (E + RT_E - 1) / RT_E);
+        route_logits_tiled<<<grid, 256, 0, stream>>>(x, T, H, gate, E, logits);
+    }
+    const SelArgs a = sel_args(T, bias, cfg, idx_out, w_out, gap_out, logits);
+    const size_t smem = sel_smem(E, SEL_WARPS);
     const unsigned grid = static_cast<unsigned>((T + SEL_WARPS - 1) / SEL_WARPS);
     route_select<<<grid, SEL_WARPS * 32, smem, stream>>>(a);
+    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+bool route_fused_ok(int64_t T, int64_t H) { return T >= 1 && T <= FUSED_MAXT && H % 32 == 0; }
+
+moe_status launch_route_fused(const uint16_t *x, int64_t T, int64_t H, const float *gate,
+                              const float *bias, const moe_router_cfg *cfg, int32_t *idx_out,
+                              float *w_out, float *logits, unsigned *counter, int32_t *counts,
+                              int32_t *offsets, int32_t *list, int32_t *tok, int32_t *pos,
+                              int32_t *unique, int32_t *n_unique, uint32_t *flags,
+                              int32_t *zero_cnt, int32_t n_zero, cudaStream_t stream) {
+    FusedRouteArgs a;
+    a.x = x;
+    a.H = H;
+    a.G = gate;
+    a.logits = logits;
+    a.sel = sel_args(T, bias, cfg, idx_out, w_out, nullptr, logits);
+    a.counter = counter;
+    a.counts = counts;
+    a.offsets = offsets;
+    a.list = list;
+    a.tok = tok;
+    a.pos = pos;
+    a.unique = unique;
+    a.n_unique = n_unique;
+    a.flags = flags;
+    a.zero_cnt = zero_cnt;
+    a.n_zero = n_zero;
+    const int E = cfg->n_experts;
+    size_t smem = static_cast<size_t>(2 * T * E + RL_WARPS * 32) * sizeof(float);
+    const size_t bsm = static_cast<size_t>(E + 48) * sizeof(int);
+    if (bsm > smem) smem = bsm;
+    if (smem > 48 * 1024 &&
+        cudaFuncSetAttribute(route_fused_small, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    route_fused_small<<<E, RL_WARPS * 32, smem, stream>>>(a);
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 

@@ -89,3 +89,11 @@ def test_workspace_sizes_grow_with_batch(so):
     b = m.moe_layer_workspace_bytes(32, 6144, 2048, cfg)
     assert 0 < a < b
     assert L.moe_expert_ffn_workspace_bytes(4, 6144, 2048) >= 256 + 4 * 2048 * 4
+
+
+def test_library_has_no_unresolved_internal_symbols(so):
+    """Every internal (namespace moe) function the library calls is defined in it."""
+    import subprocess
+    from int4_routed_expert_route_b200 import build
+    out = subprocess.run(["nm", "-u", build.LIB], capture_output=True, text=True).stdout
+    assert "_ZN3moe" not in out

@@ -49,7 +49,7 @@ def test_noalloc_rejects_oversized_request(lib):
     rc = lib.router_cfg(cfg.E, cfg.k, cfg.n_group, cfg.topk_group, cfg.rsf)
     limit = L.moe_route_noalloc_max_scratch_bytes()
     assert limit == 4 << 20
-    T = 4096  # 4096 x 256 x 8 B of partial logits > 4 MiB
+    T = 8192  # 8192 x 256 x 4 B of fp32 logits > 4 MiB
     assert lib.moe_route_workspace_bytes(T, cfg.H, rc) - 256 > limit
     fake = ctypes.c_void_p(0x100000)
     st = L.moe_route_topk_noalloc(fake, T, cfg.H, fake, fake, ctypes.byref(rc), fake, fake, None,
