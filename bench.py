@@ -134,14 +134,28 @@ def build_layer(cfg, layer=0, dev="cuda"):
                 expert_bytes=experts[0].nbytes())
 
 
+WORKLOADS = {
+    "decode": syn.DECODE,
+    "prefill": syn.PREFILL,
+    "small_batch": syn.SMALL_BATCH.with_(T=32),
+}
+
+
+def workload_name(cfg):
+    return (f"{cfg.name}: T={cfg.T} per step, H={cfg.H} I={cfg.I} E={cfg.E}+1 shared "
+            f"top-{cfg.k} n_group={cfg.n_group} topk_group={cfg.topk_group} rsf={cfg.rsf} "
+            f"int{cfg.bits}, router bias {cfg.bias_kind}")
+
+
 def run_ours(args, world, rank):
-    cfg = syn.DECODE
+    cfg = WORKLOADS[args.workload]
     T = cfg.T
     dev = torch.device("cuda")
     L = build_layer(cfg)
     stream = torch.cuda.current_stream()
     K, W = args.steps, args.warmup
     xs = syn.activations((K + W) * T, cfg.H, 1 + 1000003 * rank, dev).view(K + W, T, cfg.H)
+    idx_buf = torch.empty((K + W, T, cfg.k), dtype=torch.int32, device=dev)
     y = torch.empty((T, cfg.H), dtype=torch.float32, device=dev)
     ws = lib.Workspace(lib.moe_layer_workspace_bytes(T, cfg.H, cfg.I, L["rc"]), dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
@@ -154,7 +168,7 @@ def run_ours(args, world, rank):
 
     def step(i, events=None):
         lib.moe_layer_forward(xs[i], L["gate"], L["bias"], L["rc"], L["table"], L["shared"],
-                              cfg.bits, y=y, ws=ws, events=events)
+                              cfg.bits, y=y, ws=ws, events=events, idx_out=idx_buf[i])
 
     # The timed loop runs as one CUDA graph (flush + layer per step, events
     # inside), so host-side launch overhead does not leak into device time.
@@ -213,14 +227,33 @@ def run_ours(args, world, rank):
 
     peaks, peak_kind = measured_peaks()
     H, I = cfg.H, cfg.I
-    unique = cfg.k + 1  # T = 1: k distinct routed experts + the shared expert
-    gu_bytes = unique * 2 * (I * H // 2 + I * 4)        # gate + up nibbles and scales
-    dn_bytes = unique * (H * I // 2 + H * 4)
-    expert_bytes_step = gu_bytes + dn_bytes
-    gu_ms = float(np.mean(stage_ms[:, 2]))
-    achieved = gu_bytes / (gu_ms * 1e-3) / 1e9
+    idx_np = idx_buf[W:].cpu().numpy()
+    uniq = np.array([len(np.unique(r[r >= 0])) for r in idx_np])  # unique routed experts per step
+    pairs = np.array([int((r >= 0).sum()) for r in idx_np])        # routed (token, slot) pairs
+    ex_bytes = 2 * (I * H // 2 + I * 4) + (H * I // 2 + H * 4)    # one int4 expert
+    gu_bytes = (uniq + 1) * 2 * (I * H // 2 + I * 4)               # + shared expert
+    expert_bytes_step = (uniq + 1) * ex_bytes
+    gu_ms = stage_ms[:, 2]
     tokens = K * T * world
     value = tokens / (total_ms * 1e-3)
+    if T < 64:
+        kern = ("gateup_decode" if T <= 8 else "gateup_gemv") + " (int4 gate+up GEMV + SwiGLU, CUDA cores)"
+        achieved = float(np.mean(gu_bytes / (gu_ms * 1e-3))) / 1e9
+        roof = {"kernel": kern, "bound": "hbm", "achieved": round(achieved, 1),
+                "peak": peaks["hbm_gbs"], "peak_source": peak_kind, "unit": "GB/s",
+                "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": None,
+                "algorithmic_bytes_per_launch": int(np.mean(gu_bytes))}
+        launches = 3 if T <= 8 else 6
+    else:
+        kern = "tc_ffn<1> (tcgen05 int4->bf16 grouped GEMM, gate+up + SwiGLU)"
+        gu_flops = (pairs + T) * 2.0 * (2 * I) * H                  # 2 * M * N * K, gate and up
+        achieved = float(np.mean(gu_flops / (gu_ms * 1e-3))) / 1e12
+        roof = {"kernel": kern, "bound": "tensor", "achieved": round(achieved, 1),
+                "peak": peaks["bf16_tflops"], "peak_source": peak_kind + " (bf16 burst)",
+                "unit": "TFLOP/s", "frac": round(achieved / peaks["bf16_tflops"], 4),
+                "traffic": None, "algorithmic_flops_per_launch": float(np.mean(gu_flops))}
+        launches = 5
+    total_flops_step = (pairs + T) * 2.0 * 3 * I * H
     res = {
         "metric": METRIC,
         "value": round(value, 2),
@@ -234,23 +267,19 @@ def run_ours(args, world, rank):
         "vs_baseline": None,
         "dtype": "int4 weights, fp32 accumulate (bf16 activations)",
         "data": "synthetic (seeded N(0,0.02) weights quantised on device; x ~ N(0,1) bf16)",
-        "config": {"workload": "GLM-scale MoE layer decode, T=1 per step, H=6144 I=2048 "
-                               "E=256+1 shared top-8 n_group=8 topk_group=4 rsf=2.5 int4",
-                   "tokens_per_step": T, "l2": "flushed before every step (256 MB write, "
-                                                "outside the timed events)",
+        "config": {"workload": workload_name(cfg), "tokens_per_step": T,
+                   "l2": "flushed before every step (256 MB write, outside the timed events)",
                    "parallelism": f"replicas x{world}"},
-        "expert_gbs": round(expert_bytes_step / (total_ms / K * 1e-3) / 1e9, 1),
-        "expert_bytes_per_token": expert_bytes_step,
+        "expert_gbs": round(float(np.mean(expert_bytes_step)) / (total_ms / K * 1e-3) / 1e9, 1),
+        "expert_bytes_per_step": int(np.mean(expert_bytes_step)),
+        "unique_experts_per_step": float(np.mean(uniq)),
+        "layer_tflops": round(float(np.mean(total_flops_step)) / (total_ms / K * 1e-3) / 1e12, 2),
         "stage_ms_median": {n: round(float(np.median(stage_ms[:, s])), 5) for s, n in
                             enumerate(["router", "bucket", "gate_up", "down", "combine"])},
-        "roofline": {"kernel": "gateup_decode (int4 gate+up GEMV + SwiGLU)", "bound": "hbm",
-                     "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
-                     "peak_source": peak_kind, "unit": "GB/s",
-                     "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": None,
-                     "algorithmic_bytes_per_launch": gu_bytes},
+        "roofline": roof,
         "e2e": {"value": round(tokens / (e2e_ms * 1e-3), 2), "unit": "tokens/s",
                 "h2d_bytes_per_step": T * H * 2, "d2h_bytes_per_step": T * H * 4},
-        "gpu_launches": 3 * K,  # fused router+bucketing, gate/up, down+combine
+        "gpu_launches": launches * K,
         "clocks": clk,
         "load": {"quantize_s": round(L["load_s"], 3), "fp32_bytes": L["fp32_bytes"],
                  "int4_expert_bytes": L["expert_bytes"]},
@@ -344,6 +373,7 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="decode", choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--repeat", type=int, default=10,
                     help="replays of the captured timed loop (the last one is reported)")

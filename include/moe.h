@@ -232,14 +232,21 @@ MOE_API moe_status moe_expert_ffn(const uint16_t *x, int64_t T, int64_t H, int64
  *   y       [T, H] fp32, overwritten
  *   idx_out [T, k] int32 and w_out [T, k] fp32, nullable (routing decision)
  * ws: moe_layer_workspace_bytes(T, H, I, cfg) bytes.
- * Paths: small batches run the CUDA-core int4 GEMV kernels; large batches run
- * the tcgen05 tensor-core grouped GEMM (int4 dequantised to 16-bit in on-chip
- * memory).  MOE_PATH_AUTO picks by tokens per expert.
+ * Paths: batches below 64 tokens run the CUDA-core int4 GEMV kernels (T <= 8:
+ * a fused router + bucketing launch and two streaming GEMV launches); from 64
+ * tokens on, the tcgen05 tensor-core grouped GEMM (int4 codes converted to
+ * bf16 / fp16 in shared memory, fp32 accumulation in tensor memory, h kept in
+ * fp16; int4 experts and H, I multiples of 128 only).  The tensor-core path
+ * adds the expert outputs with fp32 atomics, so its y is not bitwise
+ * reproducible run to run; the CUDA-core path is.
  */
 #define MOE_PATH_AUTO 0
 #define MOE_PATH_GEMV 1
 #define MOE_PATH_TENSOR 2
 MOE_API size_t moe_layer_workspace_bytes(int64_t T, int64_t H, int64_t I, const moe_router_cfg *cfg);
+/* Workspace of moe_layer_forward_ex for a forced path (AUTO as above). */
+MOE_API size_t moe_layer_workspace_bytes_ex(int64_t T, int64_t H, int64_t I,
+                                            const moe_router_cfg *cfg, int32_t path);
 MOE_API moe_status moe_layer_forward(const uint16_t *x, int64_t T, int64_t H, int64_t I,
                              const float *gate, const float *bias, const moe_router_cfg *cfg,
                              const moe_expert *experts, const moe_expert *shared,

@@ -29,7 +29,8 @@ EXPORTS = ["moe_status_str", "moe_abi_version", "moe_workspace_init", "moe_works
            "moe_expert_ffn_workspace_bytes", "moe_expert_ffn", "moe_layer_workspace_bytes",
            "moe_layer_forward", "moe_layer_forward_ex", "moe_rmsnorm_bf16",
            "moe_stack_workspace_bytes", "moe_stack_forward",
-           "moe_route_noalloc_max_scratch_bytes", "moe_route_topk_noalloc"]
+           "moe_route_noalloc_max_scratch_bytes", "moe_route_topk_noalloc",
+           "moe_layer_workspace_bytes_ex"]
 
 
 class MoEError(RuntimeError):
@@ -79,12 +80,13 @@ def load():
     L.moe_abi_version.restype = _i32
     for name in ("moe_route_workspace_bytes", "moe_expert_ffn_workspace_bytes",
                  "moe_layer_workspace_bytes", "moe_stack_workspace_bytes",
-                 "moe_route_noalloc_max_scratch_bytes"):
+                 "moe_route_noalloc_max_scratch_bytes", "moe_layer_workspace_bytes_ex"):
         getattr(L, name).restype = _sz
     L.moe_route_workspace_bytes.argtypes = [_i64, _i64, ctypes.POINTER(moe_router_cfg)]
     L.moe_expert_ffn_workspace_bytes.argtypes = [_i64, _i64, _i64]
     L.moe_layer_workspace_bytes.argtypes = [_i64, _i64, _i64, ctypes.POINTER(moe_router_cfg)]
     L.moe_stack_workspace_bytes.argtypes = [_i64, _i64, _i64, ctypes.POINTER(moe_router_cfg)]
+    L.moe_layer_workspace_bytes_ex.argtypes = [_i64, _i64, _i64, ctypes.POINTER(moe_router_cfg), _i32]
     for name in EXPORTS:
         if name.endswith("_bytes") or name in ("moe_status_str", "moe_abi_version"):
             continue
@@ -293,8 +295,8 @@ def moe_expert_ffn(x, expert: QuantExpert, y, rows=None, row_w=None, ws=None, st
     return y
 
 
-def moe_layer_workspace_bytes(T, H, I, cfg):
-    return int(load().moe_layer_workspace_bytes(T, H, I, ctypes.byref(cfg)))
+def moe_layer_workspace_bytes(T, H, I, cfg, path=PATH_AUTO):
+    return int(load().moe_layer_workspace_bytes_ex(T, H, I, ctypes.byref(cfg), path))
 
 
 def moe_layer_forward(x, gate, bias, cfg, experts: ExpertTable, shared=None, weight_bits=4,
@@ -307,7 +309,7 @@ def moe_layer_forward(x, gate, bias, cfg, experts: ExpertTable, shared=None, wei
     if y is None:
         y = torch.empty((T, H), dtype=torch.float32, device=x.device)
     if ws is None:
-        ws = Workspace(moe_layer_workspace_bytes(T, H, I, cfg), x.device)
+        ws = Workspace(moe_layer_workspace_bytes(T, H, I, cfg, path), x.device)
     ev = None
     if events is not None:
         ev = (ctypes.c_void_p * LAYER_EVENTS)(*[e.cuda_event for e in events])

@@ -26,6 +26,12 @@ moe_status launch_route_fused(const uint16_t *, int64_t, int64_t, const float *,
                               int32_t *, int32_t *, int32_t *, int32_t *, int32_t *, int32_t *,
                               int32_t *, uint32_t *, int32_t *, int32_t, cudaStream_t);
 bool decode_ok(int64_t T, int64_t H, int64_t I, int32_t k, int32_t bits);
+bool tc_ok(int64_t H, int64_t I);
+moe_status run_tc_layer(const uint16_t *x, int64_t T, int64_t H, int64_t I, int32_t k, int32_t E,
+                        const moe_expert *experts, const moe_expert *shared, const int32_t *offsets,
+                        const int32_t *tok, const int32_t *tile_off, const int32_t *list,
+                        const float *w, void *h, float *y, unsigned *counters, uint32_t *flags,
+                        cudaStream_t stream, cudaEvent_t ev_down);
 moe_status run_decode_layer(const uint16_t *x, int64_t T, int64_t H, int64_t I, int32_t k,
                             int32_t bits, const moe_expert *experts, const moe_expert *shared,
                             const int32_t *unique, const int32_t *n_unique, const int32_t *offsets,
@@ -62,8 +68,10 @@ static bool cfg_ok(const moe_router_cfg *c) {
     return true;
 }
 
-// Largest batch the CUDA-core path takes on; larger batches use tensor cores.
+// Largest batch the CUDA-core path takes on; from kTensorMinT tokens on, AUTO
+// picks the tensor-core grouped GEMM.
 static constexpr int64_t kGemvMaxT = 4096;
+static constexpr int64_t kTensorMinT = 64;
 
 bool plan_layer(int64_t T, int64_t H, int64_t I, const moe_router_cfg *cfg, int32_t path,
                 LayerPlan *p) {
@@ -74,7 +82,8 @@ bool plan_layer(int64_t T, int64_t H, int64_t I, const moe_router_cfg *cfg, int3
     p->I = I;
     p->E = cfg->n_experts;
     p->k = cfg->top_k;
-    p->path = path == MOE_PATH_AUTO ? MOE_PATH_GEMV : path;
+    p->path = path == MOE_PATH_AUTO ? (T >= kTensorMinT && tc_ok(H, I) ? MOE_PATH_TENSOR : MOE_PATH_GEMV)
+                                    : path;
     p->route_ks = route_ks_for(T, H);
     const size_t P = static_cast<size_t>(T) * p->k;
     const size_t E = static_cast<size_t>(p->E);
@@ -93,7 +102,7 @@ bool plan_layer(int64_t T, int64_t H, int64_t I, const moe_router_cfg *cfg, int3
     p->off_nunique = o; o = up(o + 4);
     p->off_tiles = o;   o = up(o + (E + 2) * 4);
     p->off_h = o;       o = up(o + Pall * static_cast<size_t>(I) * 4);
-    p->off_yp = o;      o = up(o + Pall * static_cast<size_t>(H) * 4);
+    p->off_yp = o;      o = up(o + (p->path == MOE_PATH_GEMV ? Pall * static_cast<size_t>(H) * 4 : 0));
     p->total = o;
     return true;
 }
@@ -222,6 +231,14 @@ size_t moe_layer_workspace_bytes(int64_t T, int64_t H, int64_t I, const moe_rout
     return p.total;
 }
 
+size_t moe_layer_workspace_bytes_ex(int64_t T, int64_t H, int64_t I, const moe_router_cfg *cfg,
+                                    int32_t path) {
+    if (path != MOE_PATH_AUTO && path != MOE_PATH_GEMV && path != MOE_PATH_TENSOR) return 0;
+    LayerPlan p;
+    if (!plan_layer(T, H, I, cfg, path, &p)) return 0;
+    return p.total;
+}
+
 static void rec(cudaEvent_t *ev, int i, cudaStream_t s) {
     if (ev && ev[i]) record_stage_event(ev[i], s);
 }
@@ -241,7 +258,7 @@ moe_status moe_layer_forward_ex(const uint16_t *x, int64_t T, int64_t H, int64_t
         return MOE_ERR_INVALID_ARG;
     LayerPlan p;
     if (!plan_layer(T, H, I, cfg, path, &p)) return MOE_ERR_INVALID_ARG;
-    if (p.path == MOE_PATH_TENSOR) return MOE_ERR_UNSUPPORTED;
+    if (p.path == MOE_PATH_TENSOR && (!tc_ok(H, I) || weight_bits != 4)) return MOE_ERR_UNSUPPORTED;
     if (p.path == MOE_PATH_GEMV && T > kGemvMaxT) return MOE_ERR_UNSUPPORTED;
     if (!ws || ws_bytes < p.total || !aligned16(ws)) return MOE_ERR_WORKSPACE;
     if (T == 0) return MOE_OK;
@@ -275,6 +292,28 @@ moe_status moe_layer_forward_ex(const uint16_t *x, int64_t T, int64_t H, int64_t
         st = run_decode_layer(x, T, H, I, p.k, weight_bits, experts, shared, unique, nunique,
                               offsets, tok, pos, idx, w, h, yp, tile_cnt, y, accumulate, flags,
                               stream, events ? events[3] : nullptr);
+        if (st != MOE_OK) return st;
+        rec(events, 4, stream);
+        rec(events, 5, stream);
+        return MOE_OK;
+    }
+
+    if (p.path == MOE_PATH_TENSOR) {
+        int32_t *tile_off = reinterpret_cast<int32_t *>(base + p.off_tiles);
+        unsigned *tc_counters = reinterpret_cast<unsigned *>(base + p.off_flags + 128);
+        rec(events, 0, stream);
+        st = launch_route(x, T, H, gate, bias, cfg, idx, w, nullptr,
+                          reinterpret_cast<double *>(logits), stream);
+        if (st != MOE_OK) return st;
+        rec(events, 1, stream);
+        st = launch_bucket(idx, T, p.k, p.E, counts, offsets, list, tok, pos, unique, nunique, flags,
+                           128, tile_off, stream);
+        if (st != MOE_OK) return st;
+        rec(events, 2, stream);
+        if (!accumulate && cudaMemsetAsync(y, 0, static_cast<size_t>(T * H) * sizeof(float), stream) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        st = run_tc_layer(x, T, H, I, p.k, p.E, experts, shared, offsets, tok, tile_off, list, w,
+                          base + p.off_h, y, tc_counters, flags, stream, events ? events[3] : nullptr);
         if (st != MOE_OK) return st;
         rec(events, 4, stream);
         rec(events, 5, stream);

@@ -98,16 +98,8 @@ __device__ __forceinline__ f2 f2_make_bits(uint32_t lo, uint32_t hi) {
     asm("mov.b64 %0, {%1, %2};" : "=l"(r.v) : "r"(lo), "r"(hi));
     return r;
 }
-__device__ __forceinline__ float f2_lo(f2 a) {
-    float lo, hi;
-    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(a.v));
-    return lo;
-}
-__device__ __forceinline__ float f2_hi(f2 a) {
-    float lo, hi;
-    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(a.v));
-    return hi;
-}
+__device__ __forceinline__ float f2_lo(f2 a) { return __uint_as_float(static_cast<uint32_t>(a.v)); }
+__device__ __forceinline__ float f2_hi(f2 a) { return __uint_as_float(static_cast<uint32_t>(a.v >> 32)); }
 __device__ __forceinline__ float f2_sum(f2 a) {
     float lo, hi;
     asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(a.v));

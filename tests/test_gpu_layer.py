@@ -19,7 +19,7 @@ def run_and_check(lib, L, OL, x, path=0, sample=None, bias=None):
     bias = L.bias if bias is None else bias
     idx = torch.empty((T, cfg.k), dtype=torch.int32, device="cuda")
     w = torch.empty((T, cfg.k), dtype=torch.float32, device="cuda")
-    ws = lib.Workspace(lib.moe_layer_workspace_bytes(T, cfg.H, cfg.I, L.rcfg))
+    ws = lib.Workspace(lib.moe_layer_workspace_bytes(T, cfg.H, cfg.I, L.rcfg, path))
     y = lib.moe_layer_forward(x, L.gate, bias, L.rcfg, L.table, L.shared, L.bits, idx_out=idx,
                               w_out=w, ws=ws, path=path)
     assert ws.flags() == 0
