@@ -27,11 +27,13 @@ moe_status launch_route_fused(const uint16_t *, int64_t, int64_t, const float *,
                               int32_t *, uint32_t *, int32_t *, int32_t, cudaStream_t);
 bool decode_ok(int64_t T, int64_t H, int64_t I, int32_t k, int32_t bits);
 bool tc_ok(int64_t H, int64_t I);
+int32_t tc_tile_tokens();
+size_t tc_xs_bytes(int64_t T, int32_t k, int64_t H);
 moe_status run_tc_layer(const uint16_t *x, int64_t T, int64_t H, int64_t I, int32_t k, int32_t E,
                         const moe_expert *experts, const moe_expert *shared, const int32_t *offsets,
                         const int32_t *tok, const int32_t *tile_off, const int32_t *list,
-                        const float *w, void *h, float *y, unsigned *counters, uint32_t *flags,
-                        cudaStream_t stream, cudaEvent_t ev_down);
+                        const float *w, void *h, void *xs, float *y, unsigned *counters,
+                        uint32_t *flags, cudaStream_t stream, cudaEvent_t ev_down);
 moe_status run_decode_layer(const uint16_t *x, int64_t T, int64_t H, int64_t I, int32_t k,
                             int32_t bits, const moe_expert *experts, const moe_expert *shared,
                             const int32_t *unique, const int32_t *n_unique, const int32_t *offsets,
@@ -102,7 +104,9 @@ bool plan_layer(int64_t T, int64_t H, int64_t I, const moe_router_cfg *cfg, int3
     p->off_nunique = o; o = up(o + 4);
     p->off_tiles = o;   o = up(o + (E + 2) * 4);
     p->off_h = o;       o = up(o + Pall * static_cast<size_t>(I) * 4);
-    p->off_yp = o;      o = up(o + (p->path == MOE_PATH_GEMV ? Pall * static_cast<size_t>(H) * 4 : 0));
+    // GEMV path: per-pair down outputs; tensor path: expert-sorted copy of x
+    p->off_yp = o;      o = up(o + (p->path == MOE_PATH_GEMV ? Pall * static_cast<size_t>(H) * 4
+                                                              : tc_xs_bytes(T, p->k, H)));
     p->total = o;
     return true;
 }
@@ -307,13 +311,14 @@ moe_status moe_layer_forward_ex(const uint16_t *x, int64_t T, int64_t H, int64_t
         if (st != MOE_OK) return st;
         rec(events, 1, stream);
         st = launch_bucket(idx, T, p.k, p.E, counts, offsets, list, tok, pos, unique, nunique, flags,
-                           128, tile_off, stream);
+                           tc_tile_tokens(), tile_off, stream);
         if (st != MOE_OK) return st;
         rec(events, 2, stream);
         if (!accumulate && cudaMemsetAsync(y, 0, static_cast<size_t>(T * H) * sizeof(float), stream) != cudaSuccess)
             return MOE_ERR_CUDA;
         st = run_tc_layer(x, T, H, I, p.k, p.E, experts, shared, offsets, tok, tile_off, list, w,
-                          base + p.off_h, y, tc_counters, flags, stream, events ? events[3] : nullptr);
+                          base + p.off_h, base + p.off_yp, y, tc_counters, flags, stream,
+                          events ? events[3] : nullptr);
         if (st != MOE_OK) return st;
         rec(events, 4, stream);
         rec(events, 5, stream);

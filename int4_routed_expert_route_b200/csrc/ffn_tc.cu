@@ -3,7 +3,7 @@
 // Batch-union grouped GEMM ("Show HN: running GLM 5.2 on a slow computer",
 // implemented features: batch-union MoE, each unique expert read once and
 // applied to all positions routed to it; dequant-on-use int4 weights).  Two
-// passes, each a persistent kernel over tiles of 128 weight rows x <=128 tokens
+// passes, each a persistent kernel over tiles of 128 weight rows x <=256 tokens
 // of one expert:
 //   pass 1 (gate/up): D_g = Q_g X^T, D_u = Q_u X^T  (bf16 x bf16 -> fp32 in TMEM)
 //                     h = silu(s_g D_g) * (s_u D_u)  -> fp16 h[pair][I]
@@ -12,16 +12,21 @@
 // int4 codes are exact in bf16 and fp16, so dequantising to 16 bits adds no
 // error; the row scale is applied in the epilogue in fp32.
 //
-// Per k-step (64 columns) of a tile: the codes of the 128 weight rows arrive
-// in a 6-deep cp.async ring (32 bytes per row and matrix); the 128 threads
-// convert them (thread = row) into the canonical K-major 128B-swizzled
-// shared-memory layout; the token rows are gathered by cp.async straight into
-// the same layout, 4 steps ahead; one thread issues tcgen05.mma (M=128, N =
-// tokens rounded up to 16, K=16 x 4) and tcgen05.commit signals an mbarrier
-// that gates the reuse of the buffers two steps later.  All waits are bounded:
-// on timeout the kernel latches MOE_FLAG_WAIT_TIMEOUT, stops, frees its tensor
-// memory and returns.
+// Warp roles (192 threads, one CTA per SM):
+//   warp 0   TMA producer: one 2D tiled load per k-step brings the 256 token
+//            rows x 64 columns of the B operand into the K-major 128B-swizzled
+//            layout (pass 1 reads the expert-sorted copy of x, pass 2 reads h)
+//   warp 1   MMA issuer: tcgen05.mma kind::f16, M=128, N=tokens (mult. of 16)
+//   warps 2-5  converters / epilogue: each thread owns one weight row, streams
+//            its int4 codes through a private cp.async ring, converts them to
+//            16-bit values in the swizzled A layout, and after the tile's last
+//            MMA reads its TMEM lane for the epilogue
+// Hand-offs use mbarriers only (full/empty rings for A and B, accumulator
+// full/empty); every wait is bounded and a timeout latches
+// MOE_FLAG_WAIT_TIMEOUT, stops the CTA and frees its tensor memory.
 #include <cstring>
+
+#include <cuda.h>
 
 #include "common.cuh"
 
@@ -33,29 +38,27 @@ namespace tc {
 
 constexpr int BM = 128;       // weight rows per tile (MMA M)
 constexpr int BK = 64;        // columns per k-step (one 128-byte swizzle row)
-constexpr int NT = 128;       // max tokens per tile (MMA N)
-constexpr int THREADS = 128;  // 4 warps: producers, converters and epilogue
-constexpr int SB = 6;         // token-tile ring depth
-constexpr int PB = 4;         // token prefetch distance (steps)
-constexpr int SNB = 6;        // code-staging ring depth
-constexpr int PN = 5;         // code prefetch distance (steps)
+constexpr int NT = 256;       // max tokens per tile (MMA N, TMA box rows)
+constexpr int THREADS = 192;  // producer warp, MMA warp, 4 converter warps
+constexpr int NCONV = 128;    // converter threads (= weight rows)
+constexpr int SB = 4;         // token-tile ring depth
 constexpr int SA = 2;         // converted weight tiles (double buffer)
-constexpr int NBAR = 4;       // MMA-completion barrier ring
-constexpr uint32_t TMEM_COLS = 256;
+constexpr int SC = 4;         // per-thread code ring depth (prefetch SC-1 steps)
 
 constexpr int TILE_BYTES = BM * BK * 2;     // 16 KB: 128 rows x 128 B
-constexpr int BTILE_BYTES = NT * BK * 2;    // 16 KB
-constexpr int STAGE_NIB = BM * (BK / 2);    // 4 KB of codes per matrix per step
+constexpr int BTILE_BYTES = NT * BK * 2;    // 32 KB
 
 template <int NMAT>
 struct Smem {
-    static constexpr size_t a_off = 0;                                     // [SA][NMAT][TILE]
-    static constexpr size_t b_off = a_off + static_cast<size_t>(SA) * NMAT * TILE_BYTES;  // [SB][BTILE]
-    static constexpr size_t n_off = b_off + static_cast<size_t>(SB) * BTILE_BYTES;       // [SNB][NMAT][STAGE_NIB]
-    static constexpr size_t tok_off = n_off + static_cast<size_t>(SNB) * NMAT * STAGE_NIB;  // [NT] int32
-    static constexpr size_t bar_off = tok_off + NT * 4;                    // [NBAR] u64
-    static constexpr size_t misc_off = bar_off + NBAR * 8;                 // tmem addr, tile id, abort
-    static constexpr size_t total = misc_off + 64 + 1024;                  // + alignment slack
+    static constexpr size_t b_off = 0;                                               // [SB][BTILE]
+    static constexpr size_t a_off = b_off + static_cast<size_t>(SB) * BTILE_BYTES;   // [SA][NMAT][TILE]
+    static constexpr size_t c_off = a_off + static_cast<size_t>(SA) * NMAT * TILE_BYTES;  // [SC][NMAT][2][NCONV][16]
+    static constexpr size_t c_stage = static_cast<size_t>(NMAT) * 2 * NCONV * 16;
+    static constexpr size_t bar_off = c_off + SC * c_stage;                          // barriers
+    static constexpr size_t misc_off = bar_off + 16 * 8;                             // tmem addr, abort
+    static_assert(2 * SB + 2 * SA + 3 <= 16, "barrier area");
+    static constexpr size_t total = misc_off + 64 + 1024;                            // + alignment slack
+    static constexpr uint32_t tmem_cols = NMAT * NT;                                 // 512 or 256
 };
 
 struct TcArgs {
@@ -97,10 +100,21 @@ __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
                  : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
     return ok != 0;
 }
-// Bounded wait on a barrier phase; false on timeout (~ seconds).
+__device__ __forceinline__ uint64_t global_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+// Bounded wait on a barrier phase: false once about two seconds have passed
+// (or after 2^30 polls, whichever comes first).
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
-    for (uint32_t it = 0; it < (1u << 26); it++)
-        if (mbar_try(bar, parity)) return true;
+    if (mbar_try(bar, parity)) return true;
+    const uint64_t t0 = global_ns();
+    for (uint32_t it = 0; it < (1u << 22); it++) {
+        for (int i = 0; i < 256; i++)
+            if (mbar_try(bar, parity)) return true;
+        if (global_ns() - t0 > 2000000000ull) return false;
+    }
     return false;
 }
 
@@ -223,257 +237,383 @@ __device__ __forceinline__ bool qm_ok(const moe_qmat &m, int64_t rows, int64_t c
 }
 
 // ---------------------------------------------------------------------------
-// The persistent grouped-GEMM kernel.  PASS 1: gate/up + SwiGLU, PASS 2: down.
+// Barrier, TMA and tensor-map helpers of the warp-specialized kernel.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int32_t x, int32_t y, uint32_t bar) {
+    asm volatile("cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+                 ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar) : "memory");
+}
+
+struct TcMaps {
+    CUtensorMap b_main;    // pass 1: expert-sorted x; pass 2: h
+    CUtensorMap b_shared;  // pass 1: x (shared expert rows); pass 2: unused (copy of b_main)
+};
+
+// Per-tile facts every role derives identically.
+struct TileInfo {
+    bool ok;
+    Tile t;
+    int npad;
+    int32_t brow;                // first B row of the TMA box
+    const uint8_t *q[2];         // code matrices
+};
+
+template <int PASS>
+__device__ __forceinline__ TileInfo tile_info(const TcArgs &a, int64_t tile, int mtiles, int64_t R, int64_t K) {
+    TileInfo ti;
+    ti.ok = decode_tile(a, tile, mtiles, ti.t);
+    if (!ti.ok) return ti;
+    if (PASS == 1) {
+        const moe_qmat g = ti.t.ex->gate, u = ti.t.ex->up;
+        ti.ok = qm_ok(g, R, K) && qm_ok(u, R, K);
+        ti.q[0] = g.q;
+        ti.q[1] = u.q;
+        ti.brow = ti.t.shared ? ti.t.j0 : static_cast<int32_t>(ti.t.hrow + ti.t.j0);
+    } else {
+        const moe_qmat d = ti.t.ex->down;
+        ti.ok = qm_ok(d, R, K);
+        ti.q[0] = d.q;
+        ti.q[1] = d.q;
+        ti.brow = static_cast<int32_t>(ti.t.hrow + ti.t.j0);
+    }
+    ti.npad = (ti.t.n + 15) & ~15;
+    return ti;
+}
+
+// ---------------------------------------------------------------------------
+// The warp-specialized persistent grouped-GEMM kernel.
 // ---------------------------------------------------------------------------
 template <int PASS>
-__global__ void __launch_bounds__(THREADS, 1) tc_ffn(TcArgs a) {
+__global__ void __launch_bounds__(THREADS, 1) tc_ffn(const __grid_constant__ TcMaps maps, TcArgs a) {
     constexpr int NMAT = PASS == 1 ? 2 : 1;
     using L = Smem<NMAT>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t *a_tiles = sm + L::a_off;
     uint8_t *b_tiles = sm + L::b_off;
-    uint8_t *nib = sm + L::n_off;
-    int32_t *tok_s = reinterpret_cast<int32_t *>(sm + L::tok_off);
+    uint8_t *a_tiles = sm + L::a_off;
+    uint8_t *cstage = sm + L::c_off;
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + L::bar_off);
-    uint32_t *misc = reinterpret_cast<uint32_t *>(sm + L::misc_off);  // [0] tmem, [1] tile, [2] abort
+    uint32_t *misc = reinterpret_cast<uint32_t *>(sm + L::misc_off);  // [0] tmem, [1] abort
+    // barrier indices
+    const uint32_t B_FULL = smem_u32(&bars[0]);         // [SB]
+    const uint32_t B_EMPTY = smem_u32(&bars[SB]);       // [SB]
+    const uint32_t A_FULL = smem_u32(&bars[2 * SB]);    // [SA]
+    const uint32_t A_EMPTY = smem_u32(&bars[2 * SB + SA]);
+    const uint32_t ACC_FULL = smem_u32(&bars[2 * SB + 2 * SA]);
+    const uint32_t ACC_EMPTY = smem_u32(&bars[2 * SB + 2 * SA + 1]);
+    const uint32_t FIN = smem_u32(&bars[2 * SB + 2 * SA + 2]);
 
-    const int tid = threadIdx.x, warp = tid >> 5;
-    const int64_t K = PASS == 1 ? a.H : a.I;        // reduction length
-    const int64_t R = PASS == 1 ? a.I : a.H;        // weight rows
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int64_t K = PASS == 1 ? a.H : a.I;
+    const int64_t R = PASS == 1 ? a.I : a.H;
     const int mtiles = static_cast<int>(R / BM);
     const int KT = static_cast<int>(K / BK);
-    const int64_t rb = K / 2;                        // bytes per code row
-    const uint32_t fmt = PASS == 1 ? 1u : 0u;        // bf16 (x) or fp16 (h)
-    const uint32_t magic = PASS == 1 ? 0x43004300u : 0x64006400u;
-    const uint32_t subv = PASS == 1 ? 0x43084308u : 0x64086408u;
+    const int64_t rb = K / 2;
 
     if (tid == 0) {
-        for (int i = 0; i < NBAR; i++) mbar_init(smem_u32(&bars[i]), 1);
+        for (int i = 0; i < SB; i++) {
+            mbar_init(B_FULL + 8 * i, 1);
+            mbar_init(B_EMPTY + 8 * i, 1);
+        }
+        for (int i = 0; i < SA; i++) {
+            mbar_init(A_FULL + 8 * i, NCONV);
+            mbar_init(A_EMPTY + 8 * i, 1);
+        }
+        mbar_init(ACC_FULL, 1);
+        mbar_init(ACC_EMPTY, NCONV);
+        mbar_init(FIN, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-        misc[2] = 0;
+        misc[1] = 0;
     }
-    if (warp == 0) {
+    if (warp == 1) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
-                     ::"r"(smem_u32(&misc[0])), "r"(TMEM_COLS) : "memory");
+                     ::"r"(smem_u32(&misc[0])), "r"(L::tmem_cols) : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = misc[0];
+    volatile uint32_t *abort_flag = &misc[1];
 
     const int64_t total_chunks = static_cast<int64_t>(a.n_shared_chunks) + a.tile_off[a.E];
     const int64_t ntiles = total_chunks * mtiles;
-    uint32_t kglobal = 0;  // k-steps issued by this CTA so far (barrier phases)
-    bool abort = false;
+    auto fail = [&]() {
+        atomicOr(const_cast<uint32_t *>(abort_flag), 1u);
+        raise_flag(a.flags, MOE_FLAG_WAIT_TIMEOUT);
+    };
+    // warp-uniform view of the abort flag (keeps .sync.aligned ops converged)
+    auto aborted = [&]() { return __any_sync(0xffffffffu, *abort_flag != 0u) != 0; };
 
-    for (;;) {
-        __syncthreads();  // everyone has read the previous tile id
-        if (tid == 0) misc[1] = atomicAdd(a.tile_counter, 1u);
-        __syncthreads();
-        const int64_t tile = misc[1];
-        if (tile >= ntiles) break;
-        Tile t;
-        if (!decode_tile(a, tile, mtiles, t)) continue;
-        const moe_qmat *mats[2];
-        if (PASS == 1) {
-            mats[0] = &t.ex->gate;
-            mats[1] = &t.ex->up;
-        } else {
-            mats[0] = &t.ex->down;
-            mats[1] = &t.ex->down;
-        }
-        const uint8_t *qm[2];
-        bool ok = true;
-        for (int mi = 0; mi < NMAT; mi++) {
-            const moe_qmat m = *mats[mi];
-            ok = ok && qm_ok(m, R, K);
-            qm[mi] = m.q;
-        }
-        if (!ok) {
-            if (tid == 0) raise_flag(a.flags, MOE_FLAG_BAD_EXPERT_SHAPE);
-            continue;
-        }
-        const int npad = (t.n + 15) & ~15;
-        // token / h row indices of the tile
-        for (int j = tid; j < NT; j += THREADS) {
-            int32_t r = 0;
-            if (j < t.n) {
-                if (PASS == 1) r = t.toks ? t.toks[t.j0 + j] : t.j0 + j;
-                else r = static_cast<int32_t>(t.hrow + t.j0 + j);
-            }
-            tok_s[j] = r;
-        }
-        __syncthreads();
-
-        // producers ------------------------------------------------------
-        auto issue_b = [&](int kt) {  // token rows of k-step kt -> ring slot
-            uint8_t *bt = b_tiles + static_cast<size_t>(kt % SB) * BTILE_BYTES;
-            const uint32_t base = smem_u32(bt);
-            for (int q = tid; q < npad * 8; q += THREADS) {
-                const int j = q >> 3, c = q & 7;
-                const bool have = j < t.n;
-                const uint16_t *src;
-                if (PASS == 1) src = a.x + static_cast<int64_t>(tok_s[j]) * a.H + static_cast<int64_t>(kt) * BK + c * 8;
-                else src = reinterpret_cast<const uint16_t *>(a.h) + static_cast<int64_t>(tok_s[j]) * a.I + static_cast<int64_t>(kt) * BK + c * 8;
-                cp_async16(base + sw_off(j, c), have ? src : reinterpret_cast<const uint16_t *>(qm[0]), have ? 16u : 0u);
-            }
-        };
-        auto issue_n = [&](int kt) {  // codes of k-step kt -> staging slot
-            uint8_t *ns = nib + static_cast<size_t>(kt % SNB) * NMAT * STAGE_NIB;
-            for (int q = tid; q < NMAT * BM * 2; q += THREADS) {
-                const int mi = q / (BM * 2), r = (q >> 1) % BM, half = q & 1;
-                const uint8_t *src = qm[mi] + static_cast<int64_t>(t.m0 + r) * rb + static_cast<int64_t>(kt) * (BK / 2) + half * 16;
-                cp_async16(smem_u32(ns + mi * STAGE_NIB + r * 32 + half * 16), src, 16u);
-            }
-        };
-        // prologue: B(0..PB-1), N(0..PN-1) in PB commit groups (group j holds B(j))
-        for (int j = 0; j < PB; j++) {
-            if (j < KT) issue_b(j);
-            if (j == 0)
-                for (int q = 0; q <= PN - PB && q < KT; q++) issue_n(q);
-            else if (j + PN - PB < KT) issue_n(j + PN - PB);
-            cp_commit();
-        }
-
-        for (int kt = 0; kt < KT && !abort; kt++) {
-            const uint32_t kg = kglobal + kt;
-            // buffers of step kt-2 are reused below: its MMAs must be complete
-            if (kt >= 2) {
-                const uint32_t kp = kg - 2;
-                if (!mbar_wait(smem_u32(&bars[kp % NBAR]), (kp / NBAR) & 1)) abort = true;
-            }
-            if (__syncthreads_or(abort)) {
-                abort = true;
-                break;
-            }
-            if (kt + PB < KT) issue_b(kt + PB);
-            if (kt + PN < KT) issue_n(kt + PN);
-            cp_commit();
-            cp_wait<PB>();
-            __syncthreads();
-            // convert the codes of step kt (thread = row) into the swizzled tile
-            {
-                const int r = tid;
-                const uint8_t *ns = nib + static_cast<size_t>(kt % SNB) * NMAT * STAGE_NIB;
-                uint8_t *at = a_tiles + static_cast<size_t>(kt % SA) * NMAT * TILE_BYTES;
-#pragma unroll
-                for (int mi = 0; mi < NMAT; mi++) {
-                    const uint4 w0 = *reinterpret_cast<const uint4 *>(ns + mi * STAGE_NIB + r * 32);
-                    const uint4 w1 = *reinterpret_cast<const uint4 *>(ns + mi * STAGE_NIB + r * 32 + 16);
-                    const uint32_t wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-                    uint8_t *tile = at + mi * TILE_BYTES;
-#pragma unroll
-                    for (int c = 0; c < 8; c++)
-                        *reinterpret_cast<uint4 *>(tile + sw_off(r, c)) = codes_to_16bit(wv[c], magic, subv);
-                }
-            }
-            fence_proxy_async();
-            __syncthreads();
-            if (tid == 0) {
-                tc_fence_after();
-                const uint32_t idesc = f16_idesc(fmt, static_cast<uint32_t>(npad));
-                const uint32_t abase = smem_u32(a_tiles + static_cast<size_t>(kt % SA) * NMAT * TILE_BYTES);
-                const uint32_t bbase = smem_u32(b_tiles + static_cast<size_t>(kt % SB) * BTILE_BYTES);
-#pragma unroll
-                for (int ks = 0; ks < BK / 16; ks++) {
-                    const uint64_t bd = sw128_desc(bbase) + static_cast<uint64_t>(ks * 2);
-#pragma unroll
-                    for (int mi = 0; mi < NMAT; mi++) {
-                        const uint64_t ad = sw128_desc(abase + mi * TILE_BYTES) + static_cast<uint64_t>(ks * 2);
-                        mma_f16(tmem + mi * NT, ad, bd, idesc, (kt > 0 || ks > 0) ? 1u : 0u);
+    if (warp == 0) {
+        // ---------------- TMA producer ----------------
+        uint32_t kc = 0;
+        for (int64_t tile = blockIdx.x; tile < ntiles && !aborted(); tile += gridDim.x) {
+            const TileInfo ti = tile_info<PASS>(a, tile, mtiles, R, K);
+            if (!ti.ok) continue;
+            const CUtensorMap *map = (PASS == 1 && ti.t.shared) ? &maps.b_shared : &maps.b_main;
+            for (int kt = 0; kt < KT; kt++) {
+                if (lane == 0) {  // kc (loads issued so far) is tracked by lane 0
+                    const uint32_t slot = kc % SB;
+                    if (mbar_wait(B_EMPTY + 8 * slot, ((kc / SB) & 1) ^ 1)) {
+                        mbar_expect_tx(B_FULL + 8 * slot, BTILE_BYTES);
+                        tma_load_2d(smem_u32(b_tiles + static_cast<size_t>(slot) * BTILE_BYTES), map, kt * BK,
+                                    ti.brow, B_FULL + 8 * slot);
+                        kc++;
+                    } else {
+                        fail();
                     }
                 }
-                mma_commit(smem_u32(&bars[kg % NBAR]));
+                if (aborted()) break;
             }
+        }
+        // drain: the last load issued into each slot has landed before exit
+        if (lane == 0)
+            for (uint32_t j = kc > SB ? kc - SB : 0; j < kc; j++)
+                if (!mbar_wait(B_FULL + 8 * (j % SB), (j / SB) & 1)) raise_flag(a.flags, MOE_FLAG_WAIT_TIMEOUT);
+        __syncwarp();
+    } else if (warp == 1) {
+        // ---------------- MMA issuer ----------------
+        uint32_t kc = 0, tc = 0;
+        const uint32_t fmt = PASS == 1 ? 1u : 0u;
+        for (int64_t tile = blockIdx.x; tile < ntiles && !aborted(); tile += gridDim.x) {
+            const TileInfo ti = tile_info<PASS>(a, tile, mtiles, R, K);
+            if (!ti.ok) continue;
+            const uint32_t idesc = f16_idesc(fmt, static_cast<uint32_t>(ti.npad));
+            if (lane == 0 && !mbar_wait(ACC_EMPTY, (tc & 1) ^ 1)) fail();
+            for (int kt = 0; kt < KT && !aborted(); kt++, kc++) {
+                const uint32_t bs = kc % SB, as = kc % SA;
+                if (lane == 0) {
+                    bool okw = mbar_wait(A_FULL + 8 * as, (kc / SA) & 1);
+                    okw = okw && mbar_wait(B_FULL + 8 * bs, (kc / SB) & 1);
+                    if (!okw) {
+                        fail();
+                    } else {
+                        tc_fence_after();
+                        const uint32_t abase = smem_u32(a_tiles + static_cast<size_t>(as) * NMAT * TILE_BYTES);
+                        const uint32_t bbase = smem_u32(b_tiles + static_cast<size_t>(bs) * BTILE_BYTES);
+#pragma unroll
+                        for (int ks = 0; ks < BK / 16; ks++) {
+                            const uint64_t bd = sw128_desc(bbase) + static_cast<uint64_t>(ks * 2);
+#pragma unroll
+                            for (int mi = 0; mi < NMAT; mi++) {
+                                const uint64_t ad = sw128_desc(abase + mi * TILE_BYTES) + static_cast<uint64_t>(ks * 2);
+                                mma_f16(tmem + mi * NT, ad, bd, idesc, (kt > 0 || ks > 0) ? 1u : 0u);
+                            }
+                        }
+                        mma_commit(B_EMPTY + 8 * bs);
+                        mma_commit(A_EMPTY + 8 * as);
+                        if (kt == KT - 1) mma_commit(ACC_FULL);
+                    }
+                }
+                __syncwarp();
+            }
+            tc++;
+        }
+        // every MMA this thread issued has completed before the TMEM is freed
+        if (lane == 0) {
+            mma_commit(FIN);
+            if (!mbar_wait(FIN, 0)) raise_flag(a.flags, MOE_FLAG_WAIT_TIMEOUT);
+        }
+        __syncwarp();
+    } else {
+        // ---------------- converters / epilogue ----------------
+        const int ct = tid - 64;                       // 0..127
+        const int quarter = warp & 3;                  // TMEM lane quarter of this warp
+        const int r = quarter * 32 + lane;             // weight row within the tile
+        const uint32_t magic = PASS == 1 ? 0x43004300u : 0x64006400u;
+        const uint32_t subv = PASS == 1 ? 0x43084308u : 0x64086408u;
+        // Code prefetch cursor: runs SC-1 k-steps ahead of the conversion,
+        // across tile boundaries, through this CTA's sequence of valid tiles.
+        int64_t pf_tile = blockIdx.x;
+        int pf_kt = 0;
+        TileInfo pf;
+        pf.ok = false;
+        auto pf_seek = [&]() {
+            for (; pf_tile < ntiles; pf_tile += gridDim.x) {
+                pf = tile_info<PASS>(a, pf_tile, mtiles, R, K);
+                if (pf.ok) return;
+                if (ct == 0 && pf.t.n > 0) raise_flag(a.flags, MOE_FLAG_BAD_EXPERT_SHAPE);
+            }
+        };
+        auto pf_issue = [&](uint32_t slot) {
+            if (pf_tile < ntiles) {
+                uint8_t *st = cstage + static_cast<size_t>(slot) * L::c_stage;
+#pragma unroll
+                for (int mi = 0; mi < NMAT; mi++)
+#pragma unroll
+                    for (int hf = 0; hf < 2; hf++) {
+                        const uint8_t *src = pf.q[mi] + static_cast<int64_t>(pf.t.m0 + r) * rb +
+                                             static_cast<int64_t>(pf_kt) * (BK / 2) + hf * 16;
+                        cp_async16(smem_u32(st + ((mi * 2 + hf) * NCONV + ct) * 16), src, 16u);
+                    }
+                if (++pf_kt == KT) {
+                    pf_kt = 0;
+                    pf_tile += gridDim.x;
+                    pf_seek();
+                }
+            }
+            cp_commit();
+        };
+        pf_seek();
+        uint32_t kc = 0, tc = 0;
+        for (int j = 0; j < SC - 1; j++) pf_issue(static_cast<uint32_t>(j));
+        for (int64_t tile = blockIdx.x; tile < ntiles && !aborted(); tile += gridDim.x) {
+            const TileInfo ti = tile_info<PASS>(a, tile, mtiles, R, K);
+            if (!ti.ok) continue;
+            for (int kt = 0; kt < KT && !aborted(); kt++, kc++) {
+                pf_issue((kc + SC - 1) % SC);
+                cp_wait<SC - 1>();
+                const uint32_t as = kc % SA;
+                if (!mbar_wait(A_EMPTY + 8 * as, ((kc / SA) & 1) ^ 1)) fail();
+                const uint8_t *st = cstage + static_cast<size_t>(kc % SC) * L::c_stage;
+                uint8_t *at = a_tiles + static_cast<size_t>(as) * NMAT * TILE_BYTES;
+#pragma unroll
+                for (int mi = 0; mi < NMAT; mi++)
+#pragma unroll
+                    for (int hf = 0; hf < 2; hf++) {
+                        const uint4 wq = *reinterpret_cast<const uint4 *>(st + ((mi * 2 + hf) * NCONV + ct) * 16);
+                        const uint32_t wv[4] = {wq.x, wq.y, wq.z, wq.w};
+#pragma unroll
+                        for (int c = 0; c < 4; c++)
+                            *reinterpret_cast<uint4 *>(at + mi * TILE_BYTES + sw_off(r, hf * 4 + c)) =
+                                codes_to_16bit(wv[c], magic, subv);
+                    }
+                fence_proxy_async();
+                mbar_arrive(A_FULL + 8 * as);
+            }
+            // epilogue of this tile
+            if (!mbar_wait(ACC_FULL, tc & 1)) fail();
+            tc_fence_after();
+            const Tile &t = ti.t;
+            const int row = t.m0 + r;
+            const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+            if (!aborted()) {
+                if (PASS == 1) {
+                    const float sg = t.ex->gate.scale[row], su = t.ex->up.scale[row];
+                    bool ovf = false;
+                    for (int c0 = 0; c0 < ti.npad; c0 += 32) {
+                        uint32_t g[32], u[32];
+                        tmem_ld32(lane_addr + c0, g);
+                        tmem_ld32(lane_addr + NT + c0, u);
+#pragma unroll
+                        for (int i = 0; i < 32; i++) {
+                            const int j = c0 + i;
+                            if (j < t.n) {
+                                const float gv = __uint_as_float(g[i]) * sg;
+                                const float uv = __uint_as_float(u[i]) * su;
+                                const float hv = silu(gv) * uv;
+                                ovf |= !(fabsf(hv) <= 65504.0f);
+                                a.h[(t.hrow + t.j0 + j) * a.I + row] = __float2half_rn(hv);
+                            }
+                        }
+                    }
+                    if (ovf) raise_flag(a.flags, MOE_FLAG_FP16_OVERFLOW);
+                } else {
+                    const float sd = t.ex->down.scale[row];
+                    for (int c0 = 0; c0 < ti.npad; c0 += 32) {
+                        uint32_t d[32];
+                        tmem_ld32(lane_addr + c0, d);
+#pragma unroll
+                        for (int i = 0; i < 32; i++) {
+                            const int j = c0 + i;
+                            if (j < t.n) {
+                                const int64_t hr = t.hrow + t.j0 + j;
+                                const int64_t tk = t.shared ? (t.j0 + j) : a.tok[hr];
+                                const float wgt = t.shared ? 1.0f : a.w[a.list[hr]];
+                                atomicAdd(a.y + tk * a.H + row, wgt * (__uint_as_float(d[i]) * sd));
+                            }
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(ACC_EMPTY);
+            tc++;
         }
         cp_wait_all();
-        if (abort) break;
-        // wait for the last k-step's MMAs (they complete in issue order)
-        {
-            const uint32_t kl = kglobal + KT - 1;
-            if (!mbar_wait(smem_u32(&bars[kl % NBAR]), (kl / NBAR) & 1)) abort = true;
-        }
-        if (__syncthreads_or(abort)) {
-            abort = true;
-            break;
-        }
-        kglobal += KT;
-        tc_fence_after();
-
-        // epilogue: thread = weight row m0 + tid (TMEM lane tid)
-        const int row = t.m0 + tid;
-        const uint32_t lane_addr = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-        if (PASS == 1) {
-            const float sg = t.ex->gate.scale[row], su = t.ex->up.scale[row];
-            bool ovf = false;
-            for (int c0 = 0; c0 < npad; c0 += 32) {
-                uint32_t g[32], u[32];
-                tmem_ld32(lane_addr + c0, g);
-                tmem_ld32(lane_addr + NT + c0, u);
-#pragma unroll
-                for (int i = 0; i < 32; i++) {
-                    const int j = c0 + i;
-                    if (j < t.n) {
-                        const float gv = __uint_as_float(g[i]) * sg;
-                        const float uv = __uint_as_float(u[i]) * su;
-                        const float hv = silu(gv) * uv;
-                        ovf |= !(fabsf(hv) <= 65504.0f);
-                        a.h[(t.hrow + t.j0 + j) * a.I + row] = __float2half_rn(hv);
-                    }
-                }
-            }
-            if (ovf) raise_flag(a.flags, MOE_FLAG_FP16_OVERFLOW);
-        } else {
-            const float sd = t.ex->down.scale[row];
-            for (int c0 = 0; c0 < npad; c0 += 32) {
-                uint32_t d[32];
-                tmem_ld32(lane_addr + c0, d);
-#pragma unroll
-                for (int i = 0; i < 32; i++) {
-                    const int j = c0 + i;
-                    if (j < t.n) {
-                        const int64_t hr = t.hrow + t.j0 + j;
-                        const int64_t tk = t.shared ? (t.j0 + j) : a.tok[hr];
-                        const float wgt = t.shared ? 1.0f : a.w[a.list[hr]];
-                        atomicAdd(a.y + tk * a.H + row, wgt * (__uint_as_float(d[i]) * sd));
-                    }
-                }
-            }
-        }
-        tc_fence_before();
-        __syncthreads();
     }
 
-    if (abort && tid == 0) raise_flag(a.flags, MOE_FLAG_WAIT_TIMEOUT);
-    cp_wait_all();
     tc_fence_before();
     __syncthreads();
-    if (warp == 0)
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS) : "memory");
+    if (warp == 1)
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(L::tmem_cols) : "memory");
+}
+
+// Rows of x in expert-sorted order: xs[q] = x[tok[q]] for the routed pairs.
+__global__ void gather_rows(const uint16_t *__restrict__ x, const int32_t *__restrict__ tok,
+                            const int32_t *__restrict__ n_rows, int64_t H, uint16_t *__restrict__ xs) {
+    const int64_t n = *n_rows;
+    const int64_t per = H / 8;  // 16-byte vectors per row
+    for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n * per;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int64_t q = i / per, v = i % per;
+        reinterpret_cast<uint4 *>(xs + q * H)[v] = reinterpret_cast<const uint4 *>(x + static_cast<int64_t>(tok[q]) * H)[v];
+    }
 }
 
 }  // namespace tc
 
+int32_t tc_tile_tokens() { return tc::NT; }
+
 bool tc_ok(int64_t H, int64_t I) {
     return H % tc::BM == 0 && I % tc::BM == 0 && H % tc::BK == 0 && I % tc::BK == 0 &&
-           H / tc::BK >= 1 && I / tc::BK >= 1;
+           H <= (1 << 20) && I <= (1 << 20);
 }
 
-size_t tc_h_bytes(int64_t T, int32_t k, int64_t I) {
-    return static_cast<size_t>(T * k + T) * static_cast<size_t>(I) * sizeof(__half);
+size_t tc_xs_bytes(int64_t T, int32_t k, int64_t H) {
+    return static_cast<size_t>(T * k) * static_cast<size_t>(H) * sizeof(uint16_t);
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static bool tried = false;
+    if (!tried) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+        tried = true;
+    }
+    return fn;
+}
+
+// 2D map over a row-major [rows, cols] 16-bit matrix: box of 64 columns x 256
+// rows, 128-byte swizzle (the K-major operand layout of the MMA).
+static bool make_map(CUtensorMap *m, const void *base, int64_t rows, int64_t cols, bool bf16) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn || rows <= 0) return false;
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
+    const cuuint32_t box[2] = {tc::BK, tc::NT};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
+              const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 moe_status run_tc_layer(const uint16_t *x, int64_t T, int64_t H, int64_t I, int32_t k, int32_t E,
                         const moe_expert *experts, const moe_expert *shared, const int32_t *offsets,
                         const int32_t *tok, const int32_t *tile_off, const int32_t *list,
-                        const float *w, void *h, float *y, unsigned *counters, uint32_t *flags,
-                        cudaStream_t stream, cudaEvent_t ev_down) {
+                        const float *w, void *h, void *xs, float *y, unsigned *counters,
+                        uint32_t *flags, cudaStream_t stream, cudaEvent_t ev_down) {
     using namespace tc;
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    (void)counters;
     TcArgs a;
     std::memset(&a, 0, sizeof(a));
     a.T = T;
@@ -494,13 +634,27 @@ moe_status run_tc_layer(const uint16_t *x, int64_t T, int64_t H, int64_t I, int3
     a.y = y;
     a.w = w;
     a.bits = 4;
-    if (cudaMemsetAsync(counters, 0, 2 * sizeof(unsigned), stream) != cudaSuccess) return MOE_ERR_CUDA;
+    // expert-sorted copy of x for the TMA loads of pass 1
+    {
+        const int64_t vecs = T * k * (H / 8);
+        int64_t grid = (vecs + 255) / 256;
+        if (grid > 65535) grid = 65535;
+        if (grid > 0) {
+            gather_rows<<<static_cast<unsigned>(grid), 256, 0, stream>>>(x, tok, offsets + E, H,
+                                                                         static_cast<uint16_t *>(xs));
+            if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
+        }
+    }
+    TcMaps m1, m2;
+    if (!make_map(&m1.b_main, xs, T * k, H, true) || !make_map(&m1.b_shared, x, T, H, true) ||
+        !make_map(&m2.b_main, h, T * k + T, I, false))
+        return MOE_ERR_CUDA;
+    m2.b_shared = m2.b_main;
     {
         const size_t smem = Smem<2>::total;
         if (cudaFuncSetAttribute(tc_ffn<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess)
             return MOE_ERR_CUDA;
-        a.tile_counter = counters;
-        tc_ffn<1><<<sms, THREADS, smem, stream>>>(a);
+        tc_ffn<1><<<sms, THREADS, smem, stream>>>(m1, a);
         if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
     }
     if (ev_down) record_stage_event(ev_down, stream);
@@ -508,8 +662,7 @@ moe_status run_tc_layer(const uint16_t *x, int64_t T, int64_t H, int64_t I, int3
         const size_t smem = Smem<1>::total;
         if (cudaFuncSetAttribute(tc_ffn<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess)
             return MOE_ERR_CUDA;
-        a.tile_counter = counters + 1;
-        tc_ffn<2><<<sms, THREADS, smem, stream>>>(a);
+        tc_ffn<2><<<sms, THREADS, smem, stream>>>(m2, a);
         if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
     }
     return MOE_OK;
