@@ -236,9 +236,10 @@ MOE_API moe_status moe_expert_ffn(const uint16_t *x, int64_t T, int64_t H, int64
  * a fused router + bucketing launch and two streaming GEMV launches); from 64
  * tokens on, the tcgen05 tensor-core grouped GEMM (int4 codes converted to
  * bf16 / fp16 in shared memory, fp32 accumulation in tensor memory, h kept in
- * fp16; int4 experts and H, I multiples of 128 only).  The tensor-core path
- * adds the expert outputs with fp32 atomics, so its y is not bitwise
- * reproducible run to run; the CUDA-core path is.
+ * fp16; int4 experts and H, I multiples of 128 only).  Both paths write one
+ * fp32 partial per (token, expert) pair and add the partials of a token in a
+ * fixed order, so y is bitwise reproducible run to run on either path (the two
+ * paths round differently from each other).
  */
 #define MOE_PATH_AUTO 0
 #define MOE_PATH_GEMV 1

@@ -32,7 +32,7 @@ size_t tc_xs_bytes(int64_t T, int32_t k, int64_t H);
 moe_status run_tc_layer(const uint16_t *x, int64_t T, int64_t H, int64_t I, int32_t k, int32_t E,
                         const moe_expert *experts, const moe_expert *shared, const int32_t *offsets,
                         const int32_t *tok, const int32_t *tile_off, const int32_t *list,
-                        const float *w, void *h, void *xs, float *y, unsigned *counters,
+                        const float *w, void *h, void *xs, float *yp, unsigned *counters,
                         uint32_t *flags, cudaStream_t stream, cudaEvent_t ev_down);
 moe_status run_decode_layer(const uint16_t *x, int64_t T, int64_t H, int64_t I, int32_t k,
                             int32_t bits, const moe_expert *experts, const moe_expert *shared,
@@ -104,9 +104,11 @@ bool plan_layer(int64_t T, int64_t H, int64_t I, const moe_router_cfg *cfg, int3
     p->off_nunique = o; o = up(o + 4);
     p->off_tiles = o;   o = up(o + (E + 2) * 4);
     p->off_h = o;       o = up(o + Pall * static_cast<size_t>(I) * 4);
-    // GEMV path: per-pair down outputs; tensor path: expert-sorted copy of x
-    p->off_yp = o;      o = up(o + (p->path == MOE_PATH_GEMV ? Pall * static_cast<size_t>(H) * 4
-                                                              : tc_xs_bytes(T, p->k, H)));
+    // per-pair down outputs; the tensor path first keeps its expert-sorted
+    // copy of x here (read by pass 1, dead before pass 2 writes the partials)
+    const size_t yp_bytes = Pall * static_cast<size_t>(H) * 4;
+    const size_t xs_bytes = p->path == MOE_PATH_TENSOR ? tc_xs_bytes(T, p->k, H) : 0;
+    p->off_yp = o;      o = up(o + (yp_bytes > xs_bytes ? yp_bytes : xs_bytes));
     p->total = o;
     return true;
 }
@@ -314,13 +316,13 @@ moe_status moe_layer_forward_ex(const uint16_t *x, int64_t T, int64_t H, int64_t
                            tc_tile_tokens(), tile_off, stream);
         if (st != MOE_OK) return st;
         rec(events, 2, stream);
-        if (!accumulate && cudaMemsetAsync(y, 0, static_cast<size_t>(T * H) * sizeof(float), stream) != cudaSuccess)
-            return MOE_ERR_CUDA;
         st = run_tc_layer(x, T, H, I, p.k, p.E, experts, shared, offsets, tok, tile_off, list, w,
-                          base + p.off_h, base + p.off_yp, y, tc_counters, flags, stream,
+                          base + p.off_h, base + p.off_yp, yp, tc_counters, flags, stream,
                           events ? events[3] : nullptr);
         if (st != MOE_OK) return st;
         rec(events, 4, stream);
+        st = launch_combine(y, yp, pos, w, T, H, p.k, shared != nullptr, accumulate != 0, stream);
+        if (st != MOE_OK) return st;
         rec(events, 5, stream);
         return MOE_OK;
     }

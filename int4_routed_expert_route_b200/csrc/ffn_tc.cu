@@ -39,8 +39,9 @@ namespace tc {
 constexpr int BM = 128;       // weight rows per tile (MMA M)
 constexpr int BK = 64;        // columns per k-step (one 128-byte swizzle row)
 constexpr int NT = 256;       // max tokens per tile (MMA N, TMA box rows)
-constexpr int THREADS = 192;  // producer warp, MMA warp, 4 converter warps
+constexpr int THREADS = 320;  // producer warp, MMA warp, 4 converter warps, 4 epilogue warps
 constexpr int NCONV = 128;    // converter threads (= weight rows)
+constexpr int NEPI = 128;     // epilogue threads (= TMEM lanes)
 constexpr int SB = 4;         // token-tile ring depth
 constexpr int SA = 2;         // converted weight tiles (double buffer)
 constexpr int SC = 4;         // per-thread code ring depth (prefetch SC-1 steps)
@@ -55,10 +56,11 @@ struct Smem {
     static constexpr size_t c_off = a_off + static_cast<size_t>(SA) * NMAT * TILE_BYTES;  // [SC][NMAT][2][NCONV][16]
     static constexpr size_t c_stage = static_cast<size_t>(NMAT) * 2 * NCONV * 16;
     static constexpr size_t bar_off = c_off + SC * c_stage;                          // barriers
-    static constexpr size_t misc_off = bar_off + 16 * 8;                             // tmem addr, abort
-    static_assert(2 * SB + 2 * SA + 3 <= 16, "barrier area");
+    static constexpr size_t misc_off = bar_off + 24 * 8;                             // tmem addr, abort
+    static constexpr int NACC = NMAT == 1 ? 2 : 1;  // accumulator buffers (TMEM holds 512 columns)
+    static_assert(2 * SB + 2 * SA + 2 * NACC + 1 <= 24, "barrier area");
     static constexpr size_t total = misc_off + 64 + 1024;                            // + alignment slack
-    static constexpr uint32_t tmem_cols = NMAT * NT;                                 // 512 or 256
+    static constexpr uint32_t tmem_cols = NACC * NMAT * NT;                          // 512
 };
 
 struct TcArgs {
@@ -72,7 +74,7 @@ struct TcArgs {
     uint32_t *flags;
     const uint16_t *x;  // pass 1 B operand (bf16 [T, H])
     __half *h;          // pass 1 output / pass 2 B operand (fp16 [T*k + T, I])
-    float *y;           // pass 2 output
+    float *yp;          // pass 2 output: per-pair partials [T*k + T, H], rows as h
     const float *w;     // routing weights by pair id [T*k]
     int32_t bits;       // 4 (the tensor-core path takes int4 experts)
 };
@@ -305,9 +307,10 @@ __global__ void __launch_bounds__(THREADS, 1) tc_ffn(const __grid_constant__ TcM
     const uint32_t B_EMPTY = smem_u32(&bars[SB]);       // [SB]
     const uint32_t A_FULL = smem_u32(&bars[2 * SB]);    // [SA]
     const uint32_t A_EMPTY = smem_u32(&bars[2 * SB + SA]);
-    const uint32_t ACC_FULL = smem_u32(&bars[2 * SB + 2 * SA]);
-    const uint32_t ACC_EMPTY = smem_u32(&bars[2 * SB + 2 * SA + 1]);
-    const uint32_t FIN = smem_u32(&bars[2 * SB + 2 * SA + 2]);
+    constexpr int NACC = L::NACC;
+    const uint32_t ACC_FULL = smem_u32(&bars[2 * SB + 2 * SA]);           // [NACC]
+    const uint32_t ACC_EMPTY = smem_u32(&bars[2 * SB + 2 * SA + NACC]);   // [NACC]
+    const uint32_t FIN = smem_u32(&bars[2 * SB + 2 * SA + 2 * NACC]);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int64_t K = PASS == 1 ? a.H : a.I;
@@ -325,8 +328,10 @@ __global__ void __launch_bounds__(THREADS, 1) tc_ffn(const __grid_constant__ TcM
             mbar_init(A_FULL + 8 * i, NCONV);
             mbar_init(A_EMPTY + 8 * i, 1);
         }
-        mbar_init(ACC_FULL, 1);
-        mbar_init(ACC_EMPTY, NCONV);
+        for (int i = 0; i < NACC; i++) {
+            mbar_init(ACC_FULL + 8 * i, 1);
+            mbar_init(ACC_EMPTY + 8 * i, NEPI);
+        }
         mbar_init(FIN, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         misc[1] = 0;
@@ -386,7 +391,9 @@ __global__ void __launch_bounds__(THREADS, 1) tc_ffn(const __grid_constant__ TcM
             const TileInfo ti = tile_info<PASS>(a, tile, mtiles, R, K);
             if (!ti.ok) continue;
             const uint32_t idesc = f16_idesc(fmt, static_cast<uint32_t>(ti.npad));
-            if (lane == 0 && !mbar_wait(ACC_EMPTY, (tc & 1) ^ 1)) fail();
+            const uint32_t ab = tc % NACC;
+            const uint32_t dbase = tmem + ab * NMAT * NT;
+            if (lane == 0 && !mbar_wait(ACC_EMPTY + 8 * ab, ((tc / NACC) & 1) ^ 1)) fail();
             for (int kt = 0; kt < KT && !aborted(); kt++, kc++) {
                 const uint32_t bs = kc % SB, as = kc % SA;
                 if (lane == 0) {
@@ -404,12 +411,12 @@ __global__ void __launch_bounds__(THREADS, 1) tc_ffn(const __grid_constant__ TcM
 #pragma unroll
                             for (int mi = 0; mi < NMAT; mi++) {
                                 const uint64_t ad = sw128_desc(abase + mi * TILE_BYTES) + static_cast<uint64_t>(ks * 2);
-                                mma_f16(tmem + mi * NT, ad, bd, idesc, (kt > 0 || ks > 0) ? 1u : 0u);
+                                mma_f16(dbase + mi * NT, ad, bd, idesc, (kt > 0 || ks > 0) ? 1u : 0u);
                             }
                         }
                         mma_commit(B_EMPTY + 8 * bs);
                         mma_commit(A_EMPTY + 8 * as);
-                        if (kt == KT - 1) mma_commit(ACC_FULL);
+                        if (kt == KT - 1) mma_commit(ACC_FULL + 8 * ab);
                     }
                 }
                 __syncwarp();
@@ -422,11 +429,10 @@ __global__ void __launch_bounds__(THREADS, 1) tc_ffn(const __grid_constant__ TcM
             if (!mbar_wait(FIN, 0)) raise_flag(a.flags, MOE_FLAG_WAIT_TIMEOUT);
         }
         __syncwarp();
-    } else {
-        // ---------------- converters / epilogue ----------------
+    } else if (warp < 6) {
+        // ---------------- converters ----------------
         const int ct = tid - 64;                       // 0..127
-        const int quarter = warp & 3;                  // TMEM lane quarter of this warp
-        const int r = quarter * 32 + lane;             // weight row within the tile
+        const int r = ct;                              // weight row within the tile
         const uint32_t magic = PASS == 1 ? 0x43004300u : 0x64006400u;
         const uint32_t subv = PASS == 1 ? 0x43084308u : 0x64086408u;
         // Code prefetch cursor: runs SC-1 k-steps ahead of the conversion,
@@ -462,7 +468,7 @@ __global__ void __launch_bounds__(THREADS, 1) tc_ffn(const __grid_constant__ TcM
             cp_commit();
         };
         pf_seek();
-        uint32_t kc = 0, tc = 0;
+        uint32_t kc = 0;
         for (int j = 0; j < SC - 1; j++) pf_issue(static_cast<uint32_t>(j));
         for (int64_t tile = blockIdx.x; tile < ntiles && !aborted(); tile += gridDim.x) {
             const TileInfo ti = tile_info<PASS>(a, tile, mtiles, R, K);
@@ -488,15 +494,26 @@ __global__ void __launch_bounds__(THREADS, 1) tc_ffn(const __grid_constant__ TcM
                 fence_proxy_async();
                 mbar_arrive(A_FULL + 8 * as);
             }
-            // epilogue of this tile
-            if (!mbar_wait(ACC_FULL, tc & 1)) fail();
+        }
+        cp_wait_all();
+    } else {
+        // ---------------- epilogue ----------------
+        const int quarter = warp & 3;                  // TMEM lane quarter this warp may read
+        const int r = quarter * 32 + lane;             // weight row within the tile
+        uint32_t tc = 0;
+        for (int64_t tile = blockIdx.x; tile < ntiles && !aborted(); tile += gridDim.x) {
+            const TileInfo ti = tile_info<PASS>(a, tile, mtiles, R, K);
+            if (!ti.ok) continue;
+            const uint32_t ab = tc % NACC;
+            if (!mbar_wait(ACC_FULL + 8 * ab, (tc / NACC) & 1)) fail();
             tc_fence_after();
             const Tile &t = ti.t;
             const int row = t.m0 + r;
-            const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+            const uint32_t lane_addr = tmem + ab * NMAT * NT + (static_cast<uint32_t>(quarter * 32) << 16);
             if (!aborted()) {
                 if (PASS == 1) {
                     const float sg = t.ex->gate.scale[row], su = t.ex->up.scale[row];
+                    __half *hp = a.h + (t.hrow + t.j0) * a.I + row;
                     bool ovf = false;
                     for (int c0 = 0; c0 < ti.npad; c0 += 32) {
                         uint32_t g[32], u[32];
@@ -510,34 +527,29 @@ __global__ void __launch_bounds__(THREADS, 1) tc_ffn(const __grid_constant__ TcM
                                 const float uv = __uint_as_float(u[i]) * su;
                                 const float hv = silu(gv) * uv;
                                 ovf |= !(fabsf(hv) <= 65504.0f);
-                                a.h[(t.hrow + t.j0 + j) * a.I + row] = __float2half_rn(hv);
+                                hp[static_cast<int64_t>(j) * a.I] = __float2half_rn(hv);
                             }
                         }
                     }
                     if (ovf) raise_flag(a.flags, MOE_FLAG_FP16_OVERFLOW);
                 } else {
                     const float sd = t.ex->down.scale[row];
+                    float *yq = a.yp + (t.hrow + t.j0) * a.H + row;
                     for (int c0 = 0; c0 < ti.npad; c0 += 32) {
                         uint32_t d[32];
                         tmem_ld32(lane_addr + c0, d);
 #pragma unroll
                         for (int i = 0; i < 32; i++) {
                             const int j = c0 + i;
-                            if (j < t.n) {
-                                const int64_t hr = t.hrow + t.j0 + j;
-                                const int64_t tk = t.shared ? (t.j0 + j) : a.tok[hr];
-                                const float wgt = t.shared ? 1.0f : a.w[a.list[hr]];
-                                atomicAdd(a.y + tk * a.H + row, wgt * (__uint_as_float(d[i]) * sd));
-                            }
+                            if (j < t.n) yq[static_cast<int64_t>(j) * a.H] = __uint_as_float(d[i]) * sd;
                         }
                     }
                 }
             }
             tc_fence_before();
-            mbar_arrive(ACC_EMPTY);
+            mbar_arrive(ACC_EMPTY + 8 * ab);
             tc++;
         }
-        cp_wait_all();
     }
 
     tc_fence_before();
@@ -607,7 +619,7 @@ static bool make_map(CUtensorMap *m, const void *base, int64_t rows, int64_t col
 moe_status run_tc_layer(const uint16_t *x, int64_t T, int64_t H, int64_t I, int32_t k, int32_t E,
                         const moe_expert *experts, const moe_expert *shared, const int32_t *offsets,
                         const int32_t *tok, const int32_t *tile_off, const int32_t *list,
-                        const float *w, void *h, void *xs, float *y, unsigned *counters,
+                        const float *w, void *h, void *xs, float *yp, unsigned *counters,
                         uint32_t *flags, cudaStream_t stream, cudaEvent_t ev_down) {
     using namespace tc;
     int dev = 0, sms = 148;
@@ -631,7 +643,7 @@ moe_status run_tc_layer(const uint16_t *x, int64_t T, int64_t H, int64_t I, int3
     a.flags = flags;
     a.x = x;
     a.h = static_cast<__half *>(h);
-    a.y = y;
+    a.yp = yp;
     a.w = w;
     a.bits = 4;
     // expert-sorted copy of x for the TMA loads of pass 1

@@ -74,3 +74,16 @@ def test_tensor_path_accumulates(lib, glm):
     b = lib.moe_layer_forward(x, glm.gate, glm.bias, glm.rcfg, glm.table, glm.shared, 4,
                               y=base.clone(), accumulate=True, path=lib.PATH_TENSOR)
     assert torch.allclose(b, a - 0.25, rtol=0, atol=1e-4)
+
+
+def test_tensor_path_bitwise_reproducible(lib, glm):
+    """Per-pair partials combined in a fixed order: identical y run to run,
+    including experts that span several token tiles."""
+    cfg = syn.SMALL_BATCH.with_(T=1024)
+    bias = syn.router_bias(cfg, 0, "cuda")
+    x = syn.activations(1024, cfg.H, 3002, "cuda")
+    a = lib.moe_layer_forward(x, glm.gate, bias, glm.rcfg, glm.table, glm.shared, 4,
+                              path=lib.PATH_TENSOR)
+    b = lib.moe_layer_forward(x, glm.gate, bias, glm.rcfg, glm.table, glm.shared, 4,
+                              path=lib.PATH_TENSOR)
+    assert torch.equal(a, b)
