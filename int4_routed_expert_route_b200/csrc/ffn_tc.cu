@@ -12,17 +12,25 @@
 // int4 codes are exact in bf16 and fp16, so dequantising to 16 bits adds no
 // error; the row scale is applied in the epilogue in fp32.
 //
-// Warp roles (192 threads, one CTA per SM):
-//   warp 0   TMA producer: one 2D tiled load per k-step brings the 256 token
-//            rows x 64 columns of the B operand into the K-major 128B-swizzled
-//            layout (pass 1 reads the expert-sorted copy of x, pass 2 reads h)
-//   warp 1   MMA issuer: tcgen05.mma kind::f16, M=128, N=tokens (mult. of 16)
-//   warps 2-5  converters / epilogue: each thread owns one weight row, streams
-//            its int4 codes through a private cp.async ring, converts them to
-//            16-bit values in the swizzled A layout, and after the tile's last
-//            MMA reads its TMEM lane for the epilogue
-// Hand-offs use mbarriers only (full/empty rings for A and B, accumulator
-// full/empty); every wait is bounded and a timeout latches
+// Warp roles (448 threads, one CTA per SM):
+//   warp 0     TMA producer: per k-step, 2D tiled loads of 64-row boxes bring the
+//              tile's token rows x 64 columns of the B operand into the K-major
+//              128B-swizzled layout (pass 1 reads the expert-sorted copy of x,
+//              pass 2 reads h); only as many boxes as the tile has tokens
+//   warp 1     MMA issuer: tcgen05.mma kind::f16, M=128, N=tokens (mult. of 16),
+//              A operand from tensor memory, B from shared memory
+//   warps 2-9  converters: each thread owns one weight row and one matrix (pass
+//              1: gate or up) or one half of each k-step (pass 2); it streams its
+//              int4 codes through a private cp.async ring, converts them to
+//              16-bit values in registers ahead of time, and writes them into
+//              the A stage in tensor memory (tcgen05.st) once the MMA has
+//              released that stage
+//   warps 10-13 epilogue: after a tile's last MMA, read the accumulator lanes
+//              (tcgen05.ld), apply row scales, SwiGLU (pass 1) and store
+// Tensor memory (512 columns): pass 1 = gate and up accumulators (2 x 192) +
+// two A stages of 2 x 32 columns; pass 2 = two accumulators (2 x 192, so the
+// epilogue of one tile overlaps the MMAs of the next) + four A stages of 32.
+// Hand-offs use mbarriers only; every wait is bounded and a timeout latches
 // MOE_FLAG_WAIT_TIMEOUT, stops the CTA and frees its tensor memory.
 #include <cstring>
 
@@ -38,29 +46,34 @@ namespace tc {
 
 constexpr int BM = 128;       // weight rows per tile (MMA M)
 constexpr int BK = 64;        // columns per k-step (one 128-byte swizzle row)
-constexpr int NT = 256;       // max tokens per tile (MMA N, TMA box rows)
-constexpr int THREADS = 320;  // producer warp, MMA warp, 4 converter warps, 4 epilogue warps
-constexpr int NCONV = 128;    // converter threads (= weight rows)
+constexpr int NT = 192;       // max tokens per tile (MMA N)
+constexpr int BOX = 64;       // token rows per TMA box
+constexpr int THREADS = 448;  // producer, MMA, 8 converter warps, 4 epilogue warps
+constexpr int NCONV = 256;    // converter threads
 constexpr int NEPI = 128;     // epilogue threads (= TMEM lanes)
 constexpr int SB = 4;         // token-tile ring depth
-constexpr int SA = 2;         // converted weight tiles (double buffer)
-constexpr int SC = 4;         // per-thread code ring depth (prefetch SC-1 steps)
+constexpr int SC = 8;         // per-thread code ring depth (prefetch SC-1 steps)
 
-constexpr int TILE_BYTES = BM * BK * 2;     // 16 KB: 128 rows x 128 B
-constexpr int BTILE_BYTES = NT * BK * 2;    // 32 KB
+constexpr int BTILE_BYTES = NT * BK * 2;    // 24 KB: 192 rows x 128 B
+constexpr int BOX_BYTES = BOX * BK * 2;     // 8 KB
 
 template <int NMAT>
 struct Smem {
+    static constexpr int NACC = NMAT == 1 ? 2 : 1;   // accumulator buffers
+    static constexpr int SA = NMAT == 1 ? 4 : 2;     // A stages in tensor memory
+    static constexpr uint32_t a_col = NACC * NMAT * NT;          // first A column (384)
+    static constexpr uint32_t a_stage_cols = NMAT * (BK / 2);    // 32-bit columns per A stage
+    static constexpr uint32_t tmem_cols = 512;
+    static_assert(a_col + SA * a_stage_cols <= tmem_cols, "tensor memory budget");
+    static constexpr int CB = NMAT == 2 ? 32 : 16;   // code bytes (= A columns) per converter thread per k-step
+    static_assert(2 * CB == static_cast<int>(a_stage_cols), "two converter groups fill one A stage");
     static constexpr size_t b_off = 0;                                               // [SB][BTILE]
-    static constexpr size_t a_off = b_off + static_cast<size_t>(SB) * BTILE_BYTES;   // [SA][NMAT][TILE]
-    static constexpr size_t c_off = a_off + static_cast<size_t>(SA) * NMAT * TILE_BYTES;  // [SC][NMAT][2][NCONV][16]
-    static constexpr size_t c_stage = static_cast<size_t>(NMAT) * 2 * NCONV * 16;
+    static constexpr size_t c_off = b_off + static_cast<size_t>(SB) * BTILE_BYTES;   // [SC][CB/16][NCONV][16]
+    static constexpr size_t c_stage = static_cast<size_t>(CB) * NCONV;
     static constexpr size_t bar_off = c_off + SC * c_stage;                          // barriers
     static constexpr size_t misc_off = bar_off + 24 * 8;                             // tmem addr, abort
-    static constexpr int NACC = NMAT == 1 ? 2 : 1;  // accumulator buffers (TMEM holds 512 columns)
     static_assert(2 * SB + 2 * SA + 2 * NACC + 1 <= 24, "barrier area");
     static constexpr size_t total = misc_off + 64 + 1024;                            // + alignment slack
-    static constexpr uint32_t tmem_cols = NACC * NMAT * NT;                          // 512
 };
 
 struct TcArgs {
@@ -120,7 +133,6 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
     return false;
 }
 
-__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
@@ -146,6 +158,14 @@ __device__ __forceinline__ void mma_f16(uint32_t tmem_d, uint64_t adesc, uint64_
                  "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p; }"
                  ::"r"(tmem_d), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate) : "memory");
 }
+// Same with the A operand read from tensor memory (column address a_tmem,
+// lane 0): rows of A on the 128 lanes, two 16-bit K elements per column.
+__device__ __forceinline__ void mma_f16_ta(uint32_t tmem_d, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                           uint32_t accumulate) {
+    asm volatile("{ .reg .pred p; setp.ne.b32 p, %4, 0;\n\t"
+                 "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p; }"
+                 ::"r"(tmem_d), "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate) : "memory");
+}
 __device__ __forceinline__ void mma_commit(uint32_t bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
 }
@@ -163,10 +183,27 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
-// Byte offset of 16-byte chunk c of row r inside a 128B-swizzled tile.
-__device__ __forceinline__ uint32_t sw_off(int r, int c) {
-    return static_cast<uint32_t>((r >> 3) * 1024 + (r & 7) * 128 + ((c ^ (r & 7)) << 4));
+// Store 32 (16) consecutive 32-bit columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t *r) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+                 "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+                 "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};"
+                 ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]),
+                   "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]),
+                   "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]),
+                   "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]),
+                   "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+                 : "memory");
 }
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t *r) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+                 "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};"
+                 ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]),
+                   "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]),
+                   "r"(r[14]), "r"(r[15])
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // 8 int4 codes (one 32-bit word, consecutive columns) -> 8 16-bit values q
 // (exact), as 4 words of value pairs.  magic = bit pattern of 16-bit 128 (bf16)
@@ -295,21 +332,19 @@ template <int PASS>
 __global__ void __launch_bounds__(THREADS, 1) tc_ffn(const __grid_constant__ TcMaps maps, TcArgs a) {
     constexpr int NMAT = PASS == 1 ? 2 : 1;
     using L = Smem<NMAT>;
+    constexpr int NACC = L::NACC, SA = L::SA, CB = L::CB;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *b_tiles = sm + L::b_off;
-    uint8_t *a_tiles = sm + L::a_off;
     uint8_t *cstage = sm + L::c_off;
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + L::bar_off);
     uint32_t *misc = reinterpret_cast<uint32_t *>(sm + L::misc_off);  // [0] tmem, [1] abort
-    // barrier indices
-    const uint32_t B_FULL = smem_u32(&bars[0]);         // [SB]
-    const uint32_t B_EMPTY = smem_u32(&bars[SB]);       // [SB]
-    const uint32_t A_FULL = smem_u32(&bars[2 * SB]);    // [SA]
-    const uint32_t A_EMPTY = smem_u32(&bars[2 * SB + SA]);
-    constexpr int NACC = L::NACC;
-    const uint32_t ACC_FULL = smem_u32(&bars[2 * SB + 2 * SA]);           // [NACC]
-    const uint32_t ACC_EMPTY = smem_u32(&bars[2 * SB + 2 * SA + NACC]);   // [NACC]
+    const uint32_t B_FULL = smem_u32(&bars[0]);                          // [SB]
+    const uint32_t B_EMPTY = smem_u32(&bars[SB]);                        // [SB]
+    const uint32_t A_FULL = smem_u32(&bars[2 * SB]);                     // [SA]
+    const uint32_t A_EMPTY = smem_u32(&bars[2 * SB + SA]);               // [SA]
+    const uint32_t ACC_FULL = smem_u32(&bars[2 * SB + 2 * SA]);          // [NACC]
+    const uint32_t ACC_EMPTY = smem_u32(&bars[2 * SB + 2 * SA + NACC]);  // [NACC]
     const uint32_t FIN = smem_u32(&bars[2 * SB + 2 * SA + 2 * NACC]);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -363,13 +398,15 @@ __global__ void __launch_bounds__(THREADS, 1) tc_ffn(const __grid_constant__ TcM
             const TileInfo ti = tile_info<PASS>(a, tile, mtiles, R, K);
             if (!ti.ok) continue;
             const CUtensorMap *map = (PASS == 1 && ti.t.shared) ? &maps.b_shared : &maps.b_main;
+            const int nbox = (ti.npad + BOX - 1) / BOX;
             for (int kt = 0; kt < KT; kt++) {
                 if (lane == 0) {  // kc (loads issued so far) is tracked by lane 0
                     const uint32_t slot = kc % SB;
                     if (mbar_wait(B_EMPTY + 8 * slot, ((kc / SB) & 1) ^ 1)) {
-                        mbar_expect_tx(B_FULL + 8 * slot, BTILE_BYTES);
-                        tma_load_2d(smem_u32(b_tiles + static_cast<size_t>(slot) * BTILE_BYTES), map, kt * BK,
-                                    ti.brow, B_FULL + 8 * slot);
+                        mbar_expect_tx(B_FULL + 8 * slot, static_cast<uint32_t>(nbox * BOX_BYTES));
+                        const uint32_t dst = smem_u32(b_tiles + static_cast<size_t>(slot) * BTILE_BYTES);
+                        for (int bx = 0; bx < nbox; bx++)
+                            tma_load_2d(dst + bx * BOX_BYTES, map, kt * BK, ti.brow + bx * BOX, B_FULL + 8 * slot);
                         kc++;
                     } else {
                         fail();
@@ -403,16 +440,15 @@ __global__ void __launch_bounds__(THREADS, 1) tc_ffn(const __grid_constant__ TcM
                         fail();
                     } else {
                         tc_fence_after();
-                        const uint32_t abase = smem_u32(a_tiles + static_cast<size_t>(as) * NMAT * TILE_BYTES);
+                        const uint32_t abase = tmem + L::a_col + as * L::a_stage_cols;
                         const uint32_t bbase = smem_u32(b_tiles + static_cast<size_t>(bs) * BTILE_BYTES);
 #pragma unroll
                         for (int ks = 0; ks < BK / 16; ks++) {
                             const uint64_t bd = sw128_desc(bbase) + static_cast<uint64_t>(ks * 2);
 #pragma unroll
-                            for (int mi = 0; mi < NMAT; mi++) {
-                                const uint64_t ad = sw128_desc(abase + mi * TILE_BYTES) + static_cast<uint64_t>(ks * 2);
-                                mma_f16(dbase + mi * NT, ad, bd, idesc, (kt > 0 || ks > 0) ? 1u : 0u);
-                            }
+                            for (int mi = 0; mi < NMAT; mi++)
+                                mma_f16_ta(dbase + mi * NT, abase + mi * (BK / 2) + ks * 8, bd, idesc,
+                                           (kt > 0 || ks > 0) ? 1u : 0u);
                         }
                         mma_commit(B_EMPTY + 8 * bs);
                         mma_commit(A_EMPTY + 8 * as);
@@ -429,10 +465,13 @@ __global__ void __launch_bounds__(THREADS, 1) tc_ffn(const __grid_constant__ TcM
             if (!mbar_wait(FIN, 0)) raise_flag(a.flags, MOE_FLAG_WAIT_TIMEOUT);
         }
         __syncwarp();
-    } else if (warp < 6) {
+    } else if (warp < 10) {
         // ---------------- converters ----------------
-        const int ct = tid - 64;                       // 0..127
-        const int r = ct;                              // weight row within the tile
+        const int ct = tid - 64;                 // 0..255
+        const int quarter = warp & 3;            // TMEM lane quarter this warp may write
+        const int grp = (warp - 2) >> 2;         // pass 1: matrix (gate, up); pass 2: k-step half
+        const int r = quarter * 32 + lane;       // weight row within the tile
+        const uint32_t lane_bits = static_cast<uint32_t>(quarter * 32) << 16;
         const uint32_t magic = PASS == 1 ? 0x43004300u : 0x64006400u;
         const uint32_t subv = PASS == 1 ? 0x43084308u : 0x64086408u;
         // Code prefetch cursor: runs SC-1 k-steps ahead of the conversion,
@@ -451,14 +490,11 @@ __global__ void __launch_bounds__(THREADS, 1) tc_ffn(const __grid_constant__ TcM
         auto pf_issue = [&](uint32_t slot) {
             if (pf_tile < ntiles) {
                 uint8_t *st = cstage + static_cast<size_t>(slot) * L::c_stage;
+                const uint8_t *src = (PASS == 1 && grp ? pf.q[1] : pf.q[0]) + static_cast<int64_t>(pf.t.m0 + r) * rb +
+                                     static_cast<int64_t>(pf_kt) * (BK / 2) + (PASS == 1 ? 0 : grp * 16);
 #pragma unroll
-                for (int mi = 0; mi < NMAT; mi++)
-#pragma unroll
-                    for (int hf = 0; hf < 2; hf++) {
-                        const uint8_t *src = pf.q[mi] + static_cast<int64_t>(pf.t.m0 + r) * rb +
-                                             static_cast<int64_t>(pf_kt) * (BK / 2) + hf * 16;
-                        cp_async16(smem_u32(st + ((mi * 2 + hf) * NCONV + ct) * 16), src, 16u);
-                    }
+                for (int hf = 0; hf < CB / 16; hf++)
+                    cp_async16(smem_u32(st + (hf * NCONV + ct) * 16), src + hf * 16, 16u);
                 if (++pf_kt == KT) {
                     pf_kt = 0;
                     pf_tile += gridDim.x;
@@ -476,22 +512,30 @@ __global__ void __launch_bounds__(THREADS, 1) tc_ffn(const __grid_constant__ TcM
             for (int kt = 0; kt < KT && !aborted(); kt++, kc++) {
                 pf_issue((kc + SC - 1) % SC);
                 cp_wait<SC - 1>();
+                const uint8_t *st = cstage + static_cast<size_t>(kc % SC) * L::c_stage;
+                uint32_t v[CB];  // 16-bit value pairs (2 codes per byte, 2 values per column)
+#pragma unroll
+                for (int hf = 0; hf < CB / 16; hf++) {
+                    const uint4 wq = *reinterpret_cast<const uint4 *>(st + (hf * NCONV + ct) * 16);
+                    const uint32_t wv[4] = {wq.x, wq.y, wq.z, wq.w};
+#pragma unroll
+                    for (int c = 0; c < 4; c++) {
+                        const uint4 o = codes_to_16bit(wv[c], magic, subv);
+                        v[hf * 16 + c * 4 + 0] = o.x;
+                        v[hf * 16 + c * 4 + 1] = o.y;
+                        v[hf * 16 + c * 4 + 2] = o.z;
+                        v[hf * 16 + c * 4 + 3] = o.w;
+                    }
+                }
                 const uint32_t as = kc % SA;
                 if (!mbar_wait(A_EMPTY + 8 * as, ((kc / SA) & 1) ^ 1)) fail();
-                const uint8_t *st = cstage + static_cast<size_t>(kc % SC) * L::c_stage;
-                uint8_t *at = a_tiles + static_cast<size_t>(as) * NMAT * TILE_BYTES;
-#pragma unroll
-                for (int mi = 0; mi < NMAT; mi++)
-#pragma unroll
-                    for (int hf = 0; hf < 2; hf++) {
-                        const uint4 wq = *reinterpret_cast<const uint4 *>(st + ((mi * 2 + hf) * NCONV + ct) * 16);
-                        const uint32_t wv[4] = {wq.x, wq.y, wq.z, wq.w};
-#pragma unroll
-                        for (int c = 0; c < 4; c++)
-                            *reinterpret_cast<uint4 *>(at + mi * TILE_BYTES + sw_off(r, hf * 4 + c)) =
-                                codes_to_16bit(wv[c], magic, subv);
-                    }
-                fence_proxy_async();
+                __syncwarp();
+                tc_fence_after();
+                const uint32_t col = L::a_col + as * L::a_stage_cols + grp * CB;
+                if constexpr (CB == 32) tmem_st32(tmem + lane_bits + col, v);
+                else tmem_st16(tmem + lane_bits + col, v);
+                tmem_st_wait();
+                tc_fence_before();
                 mbar_arrive(A_FULL + 8 * as);
             }
         }
@@ -601,14 +645,14 @@ static EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// 2D map over a row-major [rows, cols] 16-bit matrix: box of 64 columns x 256
+// 2D map over a row-major [rows, cols] 16-bit matrix: box of 64 columns x 64
 // rows, 128-byte swizzle (the K-major operand layout of the MMA).
 static bool make_map(CUtensorMap *m, const void *base, int64_t rows, int64_t cols, bool bf16) {
     EncodeTiledFn fn = encode_fn();
     if (!fn || rows <= 0) return false;
     const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
     const cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
-    const cuuint32_t box[2] = {tc::BK, tc::NT};
+    const cuuint32_t box[2] = {tc::BK, tc::BOX};
     const cuuint32_t estr[2] = {1, 1};
     return fn(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
               const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
