@@ -99,17 +99,34 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
-def dist_setup():
+def dist_setup(backend="nccl"):
+    """One process per GPU (torchrun env vars); the layer is replicated, so the
+    only collectives are the timing barrier and the max over ranks."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    if backend == "nccl":
+        torch.cuda.set_device(local if world > 1 else 0)
     if world > 1:
         import datetime
-        torch.cuda.set_device(local)
-        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-    else:
-        torch.cuda.set_device(0)
+        torch.distributed.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
     return world, rank, local
+
+
+def ranks_max(x, world, device):
+    """Max over ranks of one float (an all-reduce on the device; identity for
+    a single rank): every multi-rank time is the slowest rank's."""
+    if world <= 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tokens_per_s(tokens_per_step, steps, world, max_ms):
+    """Whole-job throughput: the tokens all ranks processed over the slowest
+    rank's time."""
+    return tokens_per_step * steps * world / (max_ms * 1e-3)
 
 
 def build_layer(cfg, layer=0, dev="cuda"):
@@ -196,11 +213,7 @@ def run_ours(args, world, rank):
     stage_ms = np.array([[ev[i][s].elapsed_time(ev[i][s + 1]) for s in range(lib.LAYER_EVENTS - 1)]
                          for i in range(W, nsteps)])
     step_ms = stage_ms.sum(axis=1)
-    total_ms = float(step_ms.sum())
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = ranks_max(float(step_ms.sum()), world, dev)
     clk = clocks.stop()
 
     # end to end through the C ABI with host buffers: pinned x in, y out, per step
@@ -218,11 +231,7 @@ def run_ours(args, world, rank):
         hy.copy_(y, non_blocking=True)
         e2e_ev[i][1].record(stream)
     torch.cuda.synchronize()
-    e2e_ms = sum(a.elapsed_time(b) for a, b in e2e_ev[W:])
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = ranks_max(sum(a.elapsed_time(b) for a, b in e2e_ev[W:]), world, dev)
     assert ws.flags() == 0
 
     peaks, peak_kind = measured_peaks()
@@ -235,7 +244,7 @@ def run_ours(args, world, rank):
     expert_bytes_step = (uniq + 1) * ex_bytes
     gu_ms = stage_ms[:, 2]
     tokens = K * T * world
-    value = tokens / (total_ms * 1e-3)
+    value = job_tokens_per_s(T, K, world, total_ms)
     if T < 64:
         kern = ("gateup_decode" if T <= 8 else "gateup_gemv") + " (int4 gate+up GEMV + SwiGLU, CUDA cores)"
         achieved = float(np.mean(gu_bytes / (gu_ms * 1e-3))) / 1e9
@@ -277,7 +286,7 @@ def run_ours(args, world, rank):
         "stage_ms_median": {n: round(float(np.median(stage_ms[:, s])), 5) for s, n in
                             enumerate(["router", "bucket", "gate_up", "down", "combine"])},
         "roofline": roof,
-        "e2e": {"value": round(tokens / (e2e_ms * 1e-3), 2), "unit": "tokens/s",
+        "e2e": {"value": round(job_tokens_per_s(T, K, world, e2e_ms), 2), "unit": "tokens/s",
                 "h2d_bytes_per_step": T * H * 2, "d2h_bytes_per_step": T * H * 4},
         "gpu_launches": launches * K,
         "clocks": clk,

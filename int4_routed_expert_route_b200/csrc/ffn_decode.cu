@@ -76,6 +76,30 @@ __device__ __forceinline__ DSeg dec_seg(const DecodeArgs &a, int64_t s) {
     return g;
 }
 
+// Row range [r0, r1) of this block in the union row space (nseg segments of
+// seg_rows rows).  When the grid has at least one block per segment, every
+// block works inside a single segment (blocks per segment = grid / nseg, the
+// spare blocks idle): a block whose range straddled two experts would run two
+// pipelines back to back and finish long after the others.  Otherwise equal
+// contiguous ranges.
+__device__ __forceinline__ void dec_block_rows(int64_t nseg, int64_t seg_rows, int64_t &r0, int64_t &r1) {
+    const int64_t nb = gridDim.x, b = blockIdx.x;
+    if (nseg <= nb) {
+        const int64_t bps = nb / nseg;
+        const int64_t s = b / bps, piece = b % bps;
+        if (s >= nseg) {
+            r0 = r1 = 0;
+            return;
+        }
+        r0 = s * seg_rows + seg_rows * piece / bps;
+        r1 = s * seg_rows + seg_rows * (piece + 1) / bps;
+    } else {
+        const int64_t R = nseg * seg_rows;
+        r0 = R * b / nb;
+        r1 = R * (b + 1) / nb;
+    }
+}
+
 __device__ __forceinline__ bool dqmat_ok(const moe_qmat &m, int bits, int64_t rows, int64_t cols) {
     return m.q != nullptr && m.scale != nullptr && m.bits == bits && m.rows == rows && m.cols == cols;
 }
@@ -240,8 +264,8 @@ __global__ void __launch_bounds__(384, 1) gateup_decode(DecodeArgs a) {
     const int64_t chunk = static_cast<int64_t>(kw) * 32 + lane;
     const bool active = chunk * D::CH < rb;
     const int64_t col0 = chunk * D::NC;
-    const int64_t R = dec_nseg(a) * I;
-    const int64_t r0 = R * blockIdx.x / gridDim.x, r1 = R * (blockIdx.x + 1) / gridDim.x;
+    int64_t r0, r1;
+    dec_block_rows(dec_nseg(a), I, r0, r1);
 
     f2 xs[TG][NP];
     int64_t xs_seg = -1;
@@ -358,7 +382,7 @@ __global__ void __launch_bounds__(384, 1) down_decode(DecodeArgs a) {
     extern __shared__ __align__(16) uint8_t dsm_dn[];
     float *red = reinterpret_cast<float *>(dsm_dn);  // [DN_RMAX][TG][KW]
     uint8_t *ring_base = dsm_dn + static_cast<size_t>(DN_RMAX) * TG * a.kw * sizeof(float);
-    __shared__ int my_tiles[8];
+    __shared__ int my_tiles[DN_RMAX / DN_TILE + 1];
     __shared__ int n_my_tiles;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int KW = a.kw, RG = a.rg;
@@ -369,8 +393,15 @@ __global__ void __launch_bounds__(384, 1) down_decode(DecodeArgs a) {
     const bool active = chunk * D::CH < rb;
     const int64_t col0 = chunk * D::NC;
     const int64_t nseg = dec_nseg(a);
-    const int64_t R = nseg * H;
-    const int64_t r0 = R * blockIdx.x / gridDim.x, r1 = R * (blockIdx.x + 1) / gridDim.x;
+    int64_t r0, r1;
+    dec_block_rows(nseg, H, r0, r1);
+    // routing slots of the batch, staged once (T * k <= 8 * 32)
+    __shared__ int32_t s_pos[8 * 32];
+    __shared__ float s_w[8 * 32];
+    for (int i = threadIdx.x; i < T * a.k; i += blockDim.x) {
+        s_pos[i] = a.pos[i];
+        s_w[i] = a.w[i];
+    }
 
     f2 hs[TG][NP];
     for (int64_t r = r0; r < r1;) {
@@ -446,18 +477,20 @@ __global__ void __launch_bounds__(384, 1) down_decode(DecodeArgs a) {
                 __syncthreads();
             }
             // completion accounting for the 64-row tiles this sub-run touched
+            // (one thread per tile, all atomics in flight together)
             __threadfence();
+            if (threadIdx.x == 0) n_my_tiles = 0;
             __syncthreads();
-            if (threadIdx.x == 0) {
-                n_my_tiles = 0;
+            {
                 const int64_t ja = jb, je = jb + m;
-                for (int64_t c = ja / DN_TILE; c * DN_TILE < je; c++) {
+                const int64_t c = ja / DN_TILE + threadIdx.x;
+                if (c * DN_TILE < je) {
                     const int64_t lo = c * DN_TILE > ja ? c * DN_TILE : ja;
                     const int64_t hi = (c + 1) * DN_TILE < je ? (c + 1) * DN_TILE : je;
                     const int add = static_cast<int>(hi - lo);
                     const int need = static_cast<int>(nseg * DN_TILE);
                     const int old = atomicAdd(a.tile_cnt + c, add);
-                    if (old + add == need) my_tiles[n_my_tiles++] = static_cast<int>(c);
+                    if (old + add == need) my_tiles[atomicAdd(&n_my_tiles, 1)] = static_cast<int>(c);
                 }
             }
             __syncthreads();
@@ -469,12 +502,14 @@ __global__ void __launch_bounds__(384, 1) down_decode(DecodeArgs a) {
                     const int64_t t = q / DN_TILE;
                     const int64_t j = c * DN_TILE + q % DN_TILE;
                     float acc = a.accumulate ? a.y[t * H + j] : 0.0f;
+                    const float sh = a.shared ? __ldcg(a.yp + (T * a.k + t) * H + j) : 0.0f;
+#pragma unroll 8
                     for (int sl = 0; sl < a.k; sl++) {
-                        const int p = a.pos[t * a.k + sl];
-                        if (p < 0) continue;
-                        acc += a.w[t * a.k + sl] * __ldcg(a.yp + static_cast<int64_t>(p) * H + j);
+                        const int p = s_pos[t * a.k + sl];
+                        const float v = p >= 0 ? __ldcg(a.yp + static_cast<int64_t>(p) * H + j) : 0.0f;
+                        acc += s_w[t * a.k + sl] * v;
                     }
-                    if (a.shared) acc += __ldcg(a.yp + (T * a.k + t) * H + j);
+                    acc += sh;
                     a.y[t * H + j] = acc;
                 }
                 if (threadIdx.x == 0) a.tile_cnt[c] = 0;

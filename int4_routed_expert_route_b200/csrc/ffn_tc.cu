@@ -133,6 +133,12 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
     return false;
 }
 
+// Warp-wide bounded wait: lane 0 polls, the other lanes take its verdict.
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, int lane) {
+    bool ok = true;
+    if (lane == 0) ok = mbar_wait(bar, parity);
+    return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+}
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
@@ -360,12 +366,12 @@ __global__ void __launch_bounds__(THREADS, 1) tc_ffn(const __grid_constant__ TcM
             mbar_init(B_EMPTY + 8 * i, 1);
         }
         for (int i = 0; i < SA; i++) {
-            mbar_init(A_FULL + 8 * i, NCONV);
+            mbar_init(A_FULL + 8 * i, NCONV / 32);  // one arrival per converter warp
             mbar_init(A_EMPTY + 8 * i, 1);
         }
         for (int i = 0; i < NACC; i++) {
             mbar_init(ACC_FULL + 8 * i, 1);
-            mbar_init(ACC_EMPTY + 8 * i, NEPI);
+            mbar_init(ACC_EMPTY + 8 * i, NEPI / 32);  // one arrival per epilogue warp
         }
         mbar_init(FIN, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -392,75 +398,111 @@ __global__ void __launch_bounds__(THREADS, 1) tc_ffn(const __grid_constant__ TcM
     auto aborted = [&]() { return __any_sync(0xffffffffu, *abort_flag != 0u) != 0; };
 
     if (warp == 0) {
-        // ---------------- TMA producer ----------------
-        uint32_t kc = 0;
-        for (int64_t tile = blockIdx.x; tile < ntiles && !aborted(); tile += gridDim.x) {
-            const TileInfo ti = tile_info<PASS>(a, tile, mtiles, R, K);
-            if (!ti.ok) continue;
-            const CUtensorMap *map = (PASS == 1 && ti.t.shared) ? &maps.b_shared : &maps.b_main;
-            const int nbox = (ti.npad + BOX - 1) / BOX;
-            for (int kt = 0; kt < KT; kt++) {
-                if (lane == 0) {  // kc (loads issued so far) is tracked by lane 0
+        // ---------------- TMA producer (one lane) ----------------
+        if (lane == 0) {
+            uint32_t kc = 0;  // loads issued so far
+            for (int64_t tile = blockIdx.x; tile < ntiles && !*abort_flag; tile += gridDim.x) {
+                const TileInfo ti = tile_info<PASS>(a, tile, mtiles, R, K);
+                if (!ti.ok) continue;
+                const CUtensorMap *map = (PASS == 1 && ti.t.shared) ? &maps.b_shared : &maps.b_main;
+                const int nbox = (ti.npad + BOX - 1) / BOX;
+                const uint32_t tx = static_cast<uint32_t>(nbox * BOX_BYTES);
+                bool ok = true;
+                for (int kt = 0; kt < KT; kt++) {
                     const uint32_t slot = kc % SB;
-                    if (mbar_wait(B_EMPTY + 8 * slot, ((kc / SB) & 1) ^ 1)) {
-                        mbar_expect_tx(B_FULL + 8 * slot, static_cast<uint32_t>(nbox * BOX_BYTES));
-                        const uint32_t dst = smem_u32(b_tiles + static_cast<size_t>(slot) * BTILE_BYTES);
-                        for (int bx = 0; bx < nbox; bx++)
-                            tma_load_2d(dst + bx * BOX_BYTES, map, kt * BK, ti.brow + bx * BOX, B_FULL + 8 * slot);
-                        kc++;
-                    } else {
+                    if (!mbar_wait(B_EMPTY + 8 * slot, ((kc / SB) & 1) ^ 1)) {
                         fail();
+                        ok = false;
+                        break;
                     }
+                    mbar_expect_tx(B_FULL + 8 * slot, tx);
+                    const uint32_t dst = smem_u32(b_tiles + static_cast<size_t>(slot) * BTILE_BYTES);
+                    for (int bx = 0; bx < nbox; bx++)
+                        tma_load_2d(dst + bx * BOX_BYTES, map, kt * BK, ti.brow + bx * BOX, B_FULL + 8 * slot);
+                    kc++;
                 }
-                if (aborted()) break;
+                if (!ok) break;
             }
-        }
-        // drain: the last load issued into each slot has landed before exit
-        if (lane == 0)
+            // drain: the last load issued into each slot has landed before exit
             for (uint32_t j = kc > SB ? kc - SB : 0; j < kc; j++)
                 if (!mbar_wait(B_FULL + 8 * (j % SB), (j / SB) & 1)) raise_flag(a.flags, MOE_FLAG_WAIT_TIMEOUT);
+        }
         __syncwarp();
     } else if (warp == 1) {
-        // ---------------- MMA issuer ----------------
-        uint32_t kc = 0, tc = 0;
+        // ---------------- MMA issuer (one lane) ----------------
+        // The issuing thread's own instruction latency bounds back-to-back
+        // MMA issue, so its k-loop is unrolled over the ring period (4 k-steps):
+        // stage indices and most phase parities become compile-time, and every
+        // MMA operand is a loop-invariant base plus an immediate.
         const uint32_t fmt = PASS == 1 ? 1u : 0u;
-        for (int64_t tile = blockIdx.x; tile < ntiles && !aborted(); tile += gridDim.x) {
-            const TileInfo ti = tile_info<PASS>(a, tile, mtiles, R, K);
-            if (!ti.ok) continue;
-            const uint32_t idesc = f16_idesc(fmt, static_cast<uint32_t>(ti.npad));
-            const uint32_t ab = tc % NACC;
-            const uint32_t dbase = tmem + ab * NMAT * NT;
-            if (lane == 0 && !mbar_wait(ACC_EMPTY + 8 * ab, ((tc / NACC) & 1) ^ 1)) fail();
-            for (int kt = 0; kt < KT && !aborted(); kt++, kc++) {
-                const uint32_t bs = kc % SB, as = kc % SA;
-                if (lane == 0) {
-                    bool okw = mbar_wait(A_FULL + 8 * as, (kc / SA) & 1);
-                    okw = okw && mbar_wait(B_FULL + 8 * bs, (kc / SB) & 1);
-                    if (!okw) {
-                        fail();
-                    } else {
-                        tc_fence_after();
-                        const uint32_t abase = tmem + L::a_col + as * L::a_stage_cols;
-                        const uint32_t bbase = smem_u32(b_tiles + static_cast<size_t>(bs) * BTILE_BYTES);
+        const uint64_t bdesc0 = sw128_desc(smem_u32(b_tiles));
+        const uint32_t a_tm = tmem + L::a_col;
+        static_assert(SB == 4 && (SA == 2 || SA == 4), "unrolled issue assumes a 4-step ring period");
+        if (lane == 0) {
+            uint32_t kc = 0, tc = 0;
+            for (int64_t tile = blockIdx.x; tile < ntiles && !*abort_flag; tile += gridDim.x) {
+                const TileInfo ti = tile_info<PASS>(a, tile, mtiles, R, K);
+                if (!ti.ok) continue;
+                const uint32_t idesc = f16_idesc(fmt, static_cast<uint32_t>(ti.npad));
+                const uint32_t ab = tc % NACC;
+                const uint32_t dbase = tmem + ab * NMAT * NT;
+                if (!mbar_wait(ACC_EMPTY + 8 * ab, ((tc / NACC) & 1) ^ 1)) {
+                    fail();
+                    break;
+                }
+                bool ok = true;
+                if ((KT & 3) == 0 && (kc & 3) == 0) {
+                    for (int kt0 = 0; kt0 < KT && ok; kt0 += 4, kc += 4) {
+                        const uint32_t pb = (kc >> 2) & 1;  // phase parity of this block's B (and 4-stage A) uses
 #pragma unroll
-                        for (int ks = 0; ks < BK / 16; ks++) {
-                            const uint64_t bd = sw128_desc(bbase) + static_cast<uint64_t>(ks * 2);
+                        for (int u = 0; u < 4; u++) {
+                            const uint32_t as = u % SA;
+                            const uint32_t pa = SA == 4 ? pb : static_cast<uint32_t>((u >> 1) & 1);
+                            if (!mbar_wait(A_FULL + 8 * as, pa) || !mbar_wait(B_FULL + 8 * u, pb)) {
+                                fail();
+                                ok = false;
+                                break;
+                            }
+                            tc_fence_after();
+                            const uint32_t acc0 = (kt0 + u) > 0 ? 1u : 0u;
+#pragma unroll
+                            for (int ks = 0; ks < BK / 16; ks++)
+#pragma unroll
+                                for (int mi = 0; mi < NMAT; mi++)
+                                    mma_f16_ta(dbase + mi * NT, a_tm + as * L::a_stage_cols + mi * (BK / 2) + ks * 8,
+                                               bdesc0 + static_cast<uint64_t>(u * (BTILE_BYTES >> 4) + ks * 2), idesc,
+                                               ks > 0 ? 1u : acc0);
+                            mma_commit(B_EMPTY + 8 * u);
+                            mma_commit(A_EMPTY + 8 * as);
+                        }
+                    }
+                } else {
+                    // generic path (k-step counts that are not a multiple of 4)
+                    for (int kt = 0; kt < KT; kt++, kc++) {
+                        const uint32_t bs = kc % SB, as = kc % SA;
+                        if (!mbar_wait(A_FULL + 8 * as, (kc / SA) & 1) || !mbar_wait(B_FULL + 8 * bs, (kc / SB) & 1)) {
+                            fail();
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        const uint64_t bd = bdesc0 + static_cast<uint64_t>(bs * (BTILE_BYTES >> 4));
+                        const uint32_t acc0 = kt > 0 ? 1u : 0u;
+#pragma unroll
+                        for (int ks = 0; ks < BK / 16; ks++)
 #pragma unroll
                             for (int mi = 0; mi < NMAT; mi++)
-                                mma_f16_ta(dbase + mi * NT, abase + mi * (BK / 2) + ks * 8, bd, idesc,
-                                           (kt > 0 || ks > 0) ? 1u : 0u);
-                        }
+                                mma_f16_ta(dbase + mi * NT, a_tm + as * L::a_stage_cols + mi * (BK / 2) + ks * 8,
+                                           bd + static_cast<uint64_t>(ks * 2), idesc, ks > 0 ? 1u : acc0);
                         mma_commit(B_EMPTY + 8 * bs);
                         mma_commit(A_EMPTY + 8 * as);
-                        if (kt == KT - 1) mma_commit(ACC_FULL + 8 * ab);
                     }
                 }
-                __syncwarp();
+                if (!ok) break;
+                mma_commit(ACC_FULL + 8 * ab);
+                tc++;
             }
-            tc++;
-        }
-        // every MMA this thread issued has completed before the TMEM is freed
-        if (lane == 0) {
+            // every MMA this thread issued has completed before the TMEM is freed
             mma_commit(FIN);
             if (!mbar_wait(FIN, 0)) raise_flag(a.flags, MOE_FLAG_WAIT_TIMEOUT);
         }
@@ -528,15 +570,16 @@ __global__ void __launch_bounds__(THREADS, 1) tc_ffn(const __grid_constant__ TcM
                     }
                 }
                 const uint32_t as = kc % SA;
-                if (!mbar_wait(A_EMPTY + 8 * as, ((kc / SA) & 1) ^ 1)) fail();
-                __syncwarp();
+                // one lane polls, the warp follows; one arrival per warp
+                if (!warp_wait(A_EMPTY + 8 * as, ((kc / SA) & 1) ^ 1, lane)) fail();
                 tc_fence_after();
                 const uint32_t col = L::a_col + as * L::a_stage_cols + grp * CB;
                 if constexpr (CB == 32) tmem_st32(tmem + lane_bits + col, v);
                 else tmem_st16(tmem + lane_bits + col, v);
                 tmem_st_wait();
                 tc_fence_before();
-                mbar_arrive(A_FULL + 8 * as);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(A_FULL + 8 * as);
             }
         }
         cp_wait_all();
@@ -549,7 +592,7 @@ __global__ void __launch_bounds__(THREADS, 1) tc_ffn(const __grid_constant__ TcM
             const TileInfo ti = tile_info<PASS>(a, tile, mtiles, R, K);
             if (!ti.ok) continue;
             const uint32_t ab = tc % NACC;
-            if (!mbar_wait(ACC_FULL + 8 * ab, (tc / NACC) & 1)) fail();
+            if (!warp_wait(ACC_FULL + 8 * ab, (tc / NACC) & 1, lane)) fail();
             tc_fence_after();
             const Tile &t = ti.t;
             const int row = t.m0 + r;
@@ -591,7 +634,8 @@ __global__ void __launch_bounds__(THREADS, 1) tc_ffn(const __grid_constant__ TcM
                 }
             }
             tc_fence_before();
-            mbar_arrive(ACC_EMPTY + 8 * ab);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(ACC_EMPTY + 8 * ab);
             tc++;
         }
     }

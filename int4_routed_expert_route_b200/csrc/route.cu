@@ -33,24 +33,41 @@ __device__ __forceinline__ double dot4(float4 g, uint2 xv, double acc) {
     return acc;
 }
 
-// Block-level body: computes logits[t][e] for t < T of expert e = blockIdx.x.
+// Block-level body: computes the logits of expert e = blockIdx.x for tokens
+// t < T and returns them in lg[t] (valid in threads t < T).  Each lane issues
+// all the gate loads of a batch of RL_NB float4 chunks before any FMA, so a
+// warp has RL_NB cold HBM requests in flight instead of one.
+constexpr int RL_NB = 8;
+
 __device__ void logits_one_expert(const uint16_t *__restrict__ x, int64_t T, int64_t H,
-                                  const float *__restrict__ G, int E, float *__restrict__ logits,
-                                  double *red /* [RL_WARPS][RL_MAXT] smem */) {
+                                  const float *__restrict__ G, double *red /* [RL_WARPS][RL_MAXT] smem */,
+                                  float *lg /* [RL_MAXT] smem */) {
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
     const int e = blockIdx.x;
-    const int64_t L = H / RL_WARPS;  // H % 512 == 0 -> L % 64 == 0
+    const int64_t L = H / RL_WARPS;  // H % 32 == 0 -> L % 4 == 0 (16-byte gate chunks)
     const int64_t k0 = static_cast<int64_t>(wid) * L;
     const float *gr = G + static_cast<int64_t>(e) * H + k0;
     for (int64_t t0 = 0; t0 < T; t0 += 4) {
         double acc[4] = {0.0, 0.0, 0.0, 0.0};
-        for (int64_t j = 4 * lane; j < L; j += 128) {
-            const float4 g = *reinterpret_cast<const float4 *>(gr + j);
+        for (int64_t jb = 4 * lane; jb < L; jb += 128 * RL_NB) {
+            float4 g[RL_NB];
+#pragma unroll
+            for (int b = 0; b < RL_NB; b++) {
+                const int64_t j = jb + 128 * b;
+                g[b] = j < L ? __ldcs(reinterpret_cast<const float4 *>(gr + j)) : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
 #pragma unroll
             for (int u = 0; u < 4; u++) {
                 if (t0 + u < T) {
-                    const uint2 xv = *reinterpret_cast<const uint2 *>(x + (t0 + u) * H + k0 + j);
-                    acc[u] = dot4(g, xv, acc[u]);
+                    uint2 xv[RL_NB];
+#pragma unroll
+                    for (int b = 0; b < RL_NB; b++) {
+                        const int64_t j = jb + 128 * b;
+                        xv[b] = j < L ? *reinterpret_cast<const uint2 *>(x + (t0 + u) * H + k0 + j) : make_uint2(0u, 0u);
+                    }
+#pragma unroll
+                    for (int b = 0; b < RL_NB; b++)
+                        if (jb + 128 * b < L) acc[u] = dot4(g[b], xv[b], acc[u]);
                 }
             }
         }
@@ -64,7 +81,7 @@ __device__ void logits_one_expert(const uint16_t *__restrict__ x, int64_t T, int
     for (int64_t t = threadIdx.x; t < T; t += blockDim.x) {
         double v = 0.0;
         for (int w = 0; w < RL_WARPS; w++) v += red[w * RL_MAXT + t];
-        logits[t * E + e] = static_cast<float>(v);
+        lg[t] = static_cast<float>(v);
     }
 }
 
@@ -73,7 +90,9 @@ __global__ void __launch_bounds__(RL_WARPS * 32) route_logits_small(const uint16
                                                                     const float *__restrict__ G,
                                                                     int E, float *__restrict__ logits) {
     __shared__ double red[RL_WARPS * RL_MAXT];
-    logits_one_expert(x, T, H, G, E, logits, red);
+    __shared__ float lg[RL_MAXT];
+    logits_one_expert(x, T, H, G, red, lg);
+    for (int64_t t = threadIdx.x; t < T; t += blockDim.x) logits[t * E + blockIdx.x] = lg[t];
 }
 
 // ---------------------------------------------------------------------------
@@ -428,25 +447,33 @@ __device__ void bucket_small(const int32_t *idx, int P, int k, int E, int32_t *c
 __global__ void __launch_bounds__(RL_WARPS * 32) route_fused_small(FusedRouteArgs a) {
     extern __shared__ float dsm[];
     __shared__ double red[RL_WARPS * RL_MAXT];
+    __shared__ float lg[RL_MAXT];
     __shared__ unsigned ticket;
-    logits_one_expert(a.x, a.sel.T, a.H, a.G, a.sel.E, a.logits, red);
+    const int E = a.sel.E;
+    const int64_t T = a.sel.T;
+    // 1. this block's expert: logits, sigmoid scores and biased scores of all tokens
+    logits_one_expert(a.x, T, a.H, a.G, red, lg);
+    float *s_g = a.logits;          // scores [T][E]
+    float *b_g = a.logits + T * E;  // biased scores [T][E]
+    for (int64_t t = threadIdx.x; t < T; t += blockDim.x) {
+        const float sc = sigmoid_score(lg[t]);
+        s_g[t * E + blockIdx.x] = sc;
+        b_g[t * E + blockIdx.x] = sc + a.sel.bias[blockIdx.x];
+    }
     __threadfence();
     __syncthreads();
     if (threadIdx.x == 0) ticket = atomicAdd(a.counter, 1u);
     __syncthreads();
     if (ticket != gridDim.x - 1) return;
+    // 2. the last block: group-limited top-k of every token, then bucketing
     __threadfence();
     const int wid = threadIdx.x >> 5;
-    const int E = a.sel.E;
-    const int64_t T = a.sel.T;
     float *s_all = dsm;               // [T][E]
     float *b_all = dsm + T * E;       // [T][E]
     int *picks = reinterpret_cast<int *>(b_all + T * E);  // [8][32]
     for (int64_t i = threadIdx.x; i < T * E; i += blockDim.x) {
-        const int e = static_cast<int>(i % E);
-        const float sc = sigmoid_score(__ldcg(a.logits + i));
-        s_all[i] = sc;
-        b_all[i] = sc + a.sel.bias[e];
+        s_all[i] = __ldcg(s_g + i);
+        b_all[i] = __ldcg(b_g + i);
     }
     __syncthreads();
     for (int64_t t = wid; t < T; t += RL_WARPS)
@@ -458,10 +485,11 @@ __global__ void __launch_bounds__(RL_WARPS * 32) route_fused_small(FusedRouteArg
     if (threadIdx.x == 0) *a.counter = 0u;
 }
 
-// Scratch of the router: fp32 logits [T][E].
+// Scratch of the router: fp32 logits [T][E]; the fused small-batch router
+// keeps scores and biased scores there instead ([2][T][E]).
 size_t route_part_bytes(int64_t T, int64_t H, int E) {
     (void)H;
-    return static_cast<size_t>(T) * E * sizeof(float);
+    return static_cast<size_t>(T) * E * sizeof(float) * (T <= FUSED_MAXT ? 2 : 1);
 }
 
 int route_ks_for(int64_t T, int64_t H) {
