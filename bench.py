@@ -187,18 +187,32 @@ def run_ours(args, world, rank):
         lib.moe_layer_forward(xs[i], L["gate"], L["bias"], L["rc"], L["table"], L["shared"],
                               cfg.bits, y=y, ws=ws, events=events, idx_out=idx_buf[i])
 
-    # The timed loop runs as one CUDA graph (flush + layer per step, events
-    # inside), so host-side launch overhead does not leak into device time.
+    # The timed loop runs as one CUDA graph (flush + layer per step), so
+    # host-side launch overhead does not leak into device time.  It records
+    # only each step's start and end: an event between two of the layer's
+    # kernels would cut their programmatic-launch overlap.  A second graph of
+    # the same steps with every stage event gives the stage breakdown and the
+    # dominant kernel's duration.
     for i in range(W):
         flush.fill_(i & 0xff)
         step(i, ev[i])
     torch.cuda.synchronize()
+    ends = [[ev[i][0]] + [None] * (lib.LAYER_EVENTS - 2) + [ev[i][-1]] for i in range(nsteps)]
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph):
         for i in range(W, nsteps):
             flush.fill_(i & 0xff)
+            step(i, ends[i])
+    staged = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(staged):
+        for i in range(W, nsteps):
+            flush.fill_(i & 0xff)
             step(i, ev[i])
     torch.cuda.synchronize()
+    staged.replay()
+    torch.cuda.synchronize()
+    stage_ms = np.array([[ev[i][s].elapsed_time(ev[i][s + 1]) for s in range(lib.LAYER_EVENTS - 1)]
+                         for i in range(W, nsteps)])
     if world > 1:
         torch.distributed.barrier()
     clocks = ClockSampler(torch.cuda.current_device())
@@ -210,9 +224,7 @@ def run_ours(args, world, rank):
     torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
-    stage_ms = np.array([[ev[i][s].elapsed_time(ev[i][s + 1]) for s in range(lib.LAYER_EVENTS - 1)]
-                         for i in range(W, nsteps)])
-    step_ms = stage_ms.sum(axis=1)
+    step_ms = np.array([ev[i][0].elapsed_time(ev[i][-1]) for i in range(W, nsteps)])
     total_ms = ranks_max(float(step_ms.sum()), world, dev)
     clk = clocks.stop()
 

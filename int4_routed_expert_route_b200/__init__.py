@@ -312,7 +312,7 @@ def moe_layer_forward(x, gate, bias, cfg, experts: ExpertTable, shared=None, wei
         ws = Workspace(moe_layer_workspace_bytes(T, H, I, cfg, path), x.device)
     ev = None
     if events is not None:
-        ev = (ctypes.c_void_p * LAYER_EVENTS)(*[e.cuda_event for e in events])
+        ev = (ctypes.c_void_p * LAYER_EVENTS)(*[e.cuda_event if e is not None else None for e in events])
     rc = load().moe_layer_forward_ex(_ptr(x), T, H, I, _ptr(gate), _ptr(bias), ctypes.byref(cfg),
                                      experts.ptr(), shared.ptr() if shared is not None else None,
                                      weight_bits, _ptr(y), _ptr(idx_out), _ptr(w_out), ws.ptr(),

@@ -264,6 +264,8 @@ __global__ void __launch_bounds__(384, 1) gateup_decode(DecodeArgs a) {
     const int64_t chunk = static_cast<int64_t>(kw) * 32 + lane;
     const bool active = chunk * D::CH < rb;
     const int64_t col0 = chunk * D::NC;
+    griddep_wait();    // routing of this batch (previous kernel)
+    griddep_launch();  // the down kernel may start its weight prologue
     int64_t r0, r1;
     dec_block_rows(dec_nseg(a), I, r0, r1);
 
@@ -404,6 +406,7 @@ __global__ void __launch_bounds__(384, 1) down_decode(DecodeArgs a) {
     }
 
     f2 hs[TG][NP];
+    bool h_ready = false;  // h comes from the gate/up kernel: wait before the first read
     for (int64_t r = r0; r < r1;) {
         const int64_t s = r / H;
         const int64_t run_end = min(r1, (s + 1) * H);
@@ -416,11 +419,6 @@ __global__ void __launch_bounds__(384, 1) down_decode(DecodeArgs a) {
             const int m = static_cast<int>(run_end - r - sub < DN_RMAX ? run_end - r - sub : DN_RMAX);
             const int64_t jb = j_begin + sub;
             for (int64_t t0 = 0; ok && t0 < g.n_tok; t0 += TG) {
-#pragma unroll
-                for (int t = 0; t < TG; t++) {
-                    const bool have = active && t0 + t < g.n_tok;
-                    load_act<BITS, float>(a.h + (g.hrow + (have ? t0 + t : 0)) * I + col0, have, hs[t]);
-                }
                 const int nmy = rg < m ? (m - rg + RG - 1) / RG : 0;
                 const int nsteps = (nmy + U - 1) / U;
                 uint8_t *ring = ring_base + static_cast<size_t>(warp) * (DN_S * U * 32 * D::CH);
@@ -438,6 +436,15 @@ __global__ void __launch_bounds__(384, 1) down_decode(DecodeArgs a) {
                 };
 #pragma unroll
                 for (int st = 0; st < DN_S - 1; st++) issue(st);
+                if (!h_ready) {
+                    griddep_wait();
+                    h_ready = true;
+                }
+#pragma unroll
+                for (int t = 0; t < TG; t++) {
+                    const bool have = active && t0 + t < g.n_tok;
+                    load_act<BITS, float>(a.h + (g.hrow + (have ? t0 + t : 0)) * I + col0, have, hs[t]);
+                }
                 for (int st = 0; st < nsteps; st++) {
                     issue(st + DN_S - 1);
                     cp_async_wait<DN_S - 1>();
@@ -496,24 +503,24 @@ __global__ void __launch_bounds__(384, 1) down_decode(DecodeArgs a) {
             __syncthreads();
             const int nt = n_my_tiles;
             if (nt > 0) __threadfence();
-            for (int i = 0; i < nt; i++) {
-                const int64_t c = my_tiles[i];
-                for (int q = threadIdx.x; q < DN_TILE * T; q += blockDim.x) {
-                    const int64_t t = q / DN_TILE;
-                    const int64_t j = c * DN_TILE + q % DN_TILE;
-                    float acc = a.accumulate ? a.y[t * H + j] : 0.0f;
-                    const float sh = a.shared ? __ldcg(a.yp + (T * a.k + t) * H + j) : 0.0f;
+            // combine every tile this sub-run completed in one pass (independent loads)
+            for (int64_t q = threadIdx.x; q < static_cast<int64_t>(nt) * DN_TILE * T; q += blockDim.x) {
+                const int64_t c = my_tiles[q / (DN_TILE * T)];
+                const int64_t rem = q % (DN_TILE * T);
+                const int64_t t = rem / DN_TILE;
+                const int64_t j = c * DN_TILE + rem % DN_TILE;
+                float acc = a.accumulate ? a.y[t * H + j] : 0.0f;
+                const float sh = a.shared ? __ldcg(a.yp + (T * a.k + t) * H + j) : 0.0f;
 #pragma unroll 8
-                    for (int sl = 0; sl < a.k; sl++) {
-                        const int p = s_pos[t * a.k + sl];
-                        const float v = p >= 0 ? __ldcg(a.yp + static_cast<int64_t>(p) * H + j) : 0.0f;
-                        acc += s_w[t * a.k + sl] * v;
-                    }
-                    acc += sh;
-                    a.y[t * H + j] = acc;
+                for (int sl = 0; sl < a.k; sl++) {
+                    const int p = s_pos[t * a.k + sl];
+                    const float v = p >= 0 ? __ldcg(a.yp + static_cast<int64_t>(p) * H + j) : 0.0f;
+                    acc += s_w[t * a.k + sl] * v;
                 }
-                if (threadIdx.x == 0) a.tile_cnt[c] = 0;
+                acc += sh;
+                a.y[t * H + j] = acc;
             }
+            if (threadIdx.x < nt) a.tile_cnt[my_tiles[threadIdx.x]] = 0;
         }
         r = run_end;
     }
@@ -557,8 +564,7 @@ static moe_status launch_decode_bits(DecodeArgs a, cudaStream_t stream, cudaEven
         if (smem > 48 * 1024 &&
             cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess)
             return MOE_ERR_CUDA;
-        kern<<<sms, threads, smem, stream>>>(g);
-        if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
+        if (launch_pdl(kern, dim3(sms), dim3(threads), smem, stream, g) != cudaSuccess) return MOE_ERR_CUDA;
     }
     if (ev_down) record_stage_event(ev_down, stream);
     {
@@ -572,8 +578,7 @@ static moe_status launch_decode_bits(DecodeArgs a, cudaStream_t stream, cudaEven
         if (smem > 48 * 1024 &&
             cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess)
             return MOE_ERR_CUDA;
-        kern<<<sms, threads, smem, stream>>>(d);
-        if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
+        if (launch_pdl(kern, dim3(sms), dim3(threads), smem, stream, d) != cudaSuccess) return MOE_ERR_CUDA;
     }
     return MOE_OK;
 }

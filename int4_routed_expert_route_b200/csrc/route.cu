@@ -451,6 +451,7 @@ __global__ void __launch_bounds__(RL_WARPS * 32) route_fused_small(FusedRouteArg
     __shared__ unsigned ticket;
     const int E = a.sel.E;
     const int64_t T = a.sel.T;
+    griddep_launch();  // the gate/up kernel's blocks may be scheduled meanwhile
     // 1. this block's expert: logits, sigmoid scores and biased scores of all tokens
     logits_one_expert(a.x, T, a.H, a.G, red, lg);
     float *s_g = a.logits;          // scores [T][E]
