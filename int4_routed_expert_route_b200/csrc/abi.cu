@@ -263,7 +263,11 @@ moe_status moe_layer_forward_ex(const uint16_t *x, int64_t T, int64_t H, int64_t
     if (!aligned16(x) || !aligned16(gate) || !aligned16(y) || !aligned16(experts))
         return MOE_ERR_INVALID_ARG;
     LayerPlan p;
-    if (!plan_layer(T, H, I, cfg, path, &p)) return MOE_ERR_INVALID_ARG;
+    // the tensor-core path takes int4 experts only: AUTO sends int8 / int2
+    // layers to the CUDA-core path at every batch size (its workspace is no
+    // larger than the one moe_layer_workspace_bytes sizes for AUTO)
+    const int32_t eff_path = (path == MOE_PATH_AUTO && weight_bits != 4) ? MOE_PATH_GEMV : path;
+    if (!plan_layer(T, H, I, cfg, eff_path, &p)) return MOE_ERR_INVALID_ARG;
     if (p.path == MOE_PATH_TENSOR && (!tc_ok(H, I) || weight_bits != 4)) return MOE_ERR_UNSUPPORTED;
     if (p.path == MOE_PATH_GEMV && T > kGemvMaxT) return MOE_ERR_UNSUPPORTED;
     if (!ws || ws_bytes < p.total || !aligned16(ws)) return MOE_ERR_WORKSPACE;

@@ -213,8 +213,9 @@ __device__ __forceinline__ float sigmoid_score(float logit) {
 }
 
 // Selection of token t by one warp from its scores s_sm[E] and biased scores
-// b_sm[E] in shared memory (b_sm is consumed); pick is 32 ints of scratch.
-__device__ void select_core(const SelArgs &a, int64_t t, const float *s_sm, float *b_sm, int *pick) {
+// b_sm[E] in shared memory (read only); pick is 32 ints of scratch.
+template <int MAXJ>  // candidate slots per lane: E <= 32 * MAXJ
+__device__ void select_core_j(const SelArgs &a, int64_t t, const float *s_sm, float *b_sm, int *pick) {
     const int lane = threadIdx.x & 31;
     const int E = a.E;
 
@@ -257,38 +258,47 @@ __device__ void select_core(const SelArgs &a, int64_t t, const float *s_sm, floa
     const bool any_dropped = ng > a.topk_group;
     const unsigned gmask = __ballot_sync(0xffffffffu, gsel);
 
-    // top-k experts of b among the kept groups, descending, ties to lower index
+    // top-k experts of b among the kept groups, descending, ties to lower index.
+    // Each lane keeps its candidates e = lane + 32 j in registers with a
+    // bitmask of the ones still selectable (kept group, not yet taken).
+    const int nj = (E + 31) >> 5;
+    float cb[MAXJ];
+    uint32_t live = 0u;
+#pragma unroll
+    for (int j = 0; j < MAXJ; j++) {
+        const int e = lane + 32 * j;
+        cb[j] = -INFINITY;
+        if (j < nj && e < E && ((gmask >> (e / gsz)) & 1u)) {
+            cb[j] = b_sm[e];
+            live |= 1u << j;
+        }
+    }
     float bk = 0.0f;
     for (int r = 0; r < a.k; r++) {
         float v = -INFINITY;
         int i = 0x7fffffff;
-        for (int e = lane; e < E; e += 32) {
-            if (!((gmask >> (e / gsz)) & 1u)) continue;
-            const float b = b_sm[e];
-            if (b > v || (b == v && e < i)) {
-                v = b;
-                i = e;
+#pragma unroll
+        for (int j = 0; j < MAXJ; j++)
+            if (((live >> j) & 1u) && (cb[j] > v || (cb[j] == v && lane + 32 * j < i))) {
+                v = cb[j];
+                i = lane + 32 * j;
             }
-        }
         warp_argmax(v, i);
         if (i >= E) i = -1;  // no candidate left (only with non-finite scores)
         if (lane == 0) pick[r] = i;
-        __syncwarp();
-        if (i >= 0 && lane == (i & 31)) b_sm[i] = -INFINITY;  // taken
-        __syncwarp();
+        if (i >= 0 && lane == (i & 31)) live &= ~(1u << (i >> 5));  // taken
         bk = v;
     }
+    __syncwarp();
     float rest = -INFINITY;
     {
         int i = 0x7fffffff;
-        for (int e = lane; e < E; e += 32) {
-            if (!((gmask >> (e / gsz)) & 1u)) continue;
-            const float b = b_sm[e];
-            if (b > rest || (b == rest && e < i)) {
-                rest = b;
-                i = e;
+#pragma unroll
+        for (int j = 0; j < MAXJ; j++)
+            if (((live >> j) & 1u) && (cb[j] > rest || (cb[j] == rest && lane + 32 * j < i))) {
+                rest = cb[j];
+                i = lane + 32 * j;
             }
-        }
         warp_argmax(rest, i);
     }
     const int cand = __popc(gmask) * gsz;
@@ -333,6 +343,12 @@ __device__ void select_core(const SelArgs &a, int64_t t, const float *s_sm, floa
             a.gap_out[t] = gap;
         }
     }
+}
+
+__device__ void select_core(const SelArgs &a, int64_t t, const float *s_sm, float *b_sm, int *pick) {
+    if (a.E <= 256) select_core_j<8>(a, t, s_sm, b_sm, pick);
+    else if (a.E <= 512) select_core_j<16>(a, t, s_sm, b_sm, pick);
+    else select_core_j<32>(a, t, s_sm, b_sm, pick);
 }
 
 // Routes token t with one warp; wsm is this warp's shared scratch of
