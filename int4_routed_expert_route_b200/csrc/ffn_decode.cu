@@ -240,8 +240,8 @@ __device__ __forceinline__ void lds_chunk(const uint8_t *p, uint32_t w[Chunk<BIT
 }
 
 constexpr int DEC_RMAX = 128;  // rows per run (shared-memory partials)
-constexpr int GU_S = 4;        // gate/up copy-ring stages
-constexpr int DN_S = 8;        // down copy-ring stages
+constexpr int GU_S = 2;        // gate/up copy-ring stages (of GU_U rows)
+constexpr int DN_S = 4;        // down copy-ring stages (of DN_U rows)
 constexpr int DN_RMAX = 512;   // rows per down run
 
 // ---------------------------------------------------------------------------
@@ -536,7 +536,7 @@ static int dec_sm_count() {
     return n;
 }
 
-static constexpr int DEC_U = 4;
+static constexpr int GU_U = 8, DN_U = 8;  // rows per ring stage
 
 bool decode_ok(int64_t T, int64_t H, int64_t I, int32_t k, int32_t bits) {
     (void)k;
@@ -559,8 +559,8 @@ static moe_status launch_decode_bits(DecodeArgs a, cudaStream_t stream, cudaEven
         g.rg = 12 / kw_gu > 0 ? 12 / kw_gu : 1;
         const int threads = 32 * g.kw * g.rg;
         const size_t smem = static_cast<size_t>(DEC_RMAX) * 2 * TG * g.kw * sizeof(float) +
-                            static_cast<size_t>(threads / 32) * GU_S * DEC_U * 2 * 32 * D::CH;
-        auto kern = gateup_decode<BITS, TG, DEC_U>;
+                            static_cast<size_t>(threads / 32) * GU_S * GU_U * 2 * 32 * D::CH;
+        auto kern = gateup_decode<BITS, TG, GU_U>;
         if (smem > 48 * 1024 &&
             cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess)
             return MOE_ERR_CUDA;
@@ -573,8 +573,8 @@ static moe_status launch_decode_bits(DecodeArgs a, cudaStream_t stream, cudaEven
         d.rg = 12 / kw_dn > 0 ? 12 / kw_dn : 1;
         const int threads = 32 * d.kw * d.rg;
         const size_t smem = static_cast<size_t>(DN_RMAX) * TG * d.kw * sizeof(float) +
-                            static_cast<size_t>(threads / 32) * DN_S * DEC_U * 32 * D::CH;
-        auto kern = down_decode<BITS, TG, DEC_U>;
+                            static_cast<size_t>(threads / 32) * DN_S * DN_U * 32 * D::CH;
+        auto kern = down_decode<BITS, TG, DN_U>;
         if (smem > 48 * 1024 &&
             cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess)
             return MOE_ERR_CUDA;

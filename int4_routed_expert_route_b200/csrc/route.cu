@@ -214,6 +214,50 @@ __device__ __forceinline__ float sigmoid_score(float logit) {
 
 // Selection of token t by one warp from its scores s_sm[E] and biased scores
 // b_sm[E] in shared memory (read only); pick is 32 ints of scratch.
+// Weights, optional top-p and the decision margin of token t from its picks
+// (one thread): w = s[idx] / sum(s[picks]) * rsf in slot order.
+__device__ void select_finish(const SelArgs &a, int64_t t, const float *s_sm, const int *pick, float bk,
+                              float rest, float last_kept, float best_dropped, bool any_dropped, int cand) {
+    const int k = a.k;
+    int32_t *idx = a.idx_out + t * k;
+    float *w = a.w_out + t * k;
+    float sum = 0.0f;
+    for (int r = 0; r < k; r++)
+        if (pick[r] >= 0) sum += s_sm[pick[r]];
+    for (int r = 0; r < k; r++) {
+        idx[r] = pick[r];
+        w[r] = pick[r] >= 0 ? (s_sm[pick[r]] / sum) * a.rsf : 0.0f;
+    }
+    if (a.topp > 0.0f && a.topp < 1.0f) {
+        // rank the slots by weight (ties keep slot order), keep the shortest
+        // prefix that reaches topp * total
+        float total = 0.0f;
+        for (int r = 0; r < k; r++) total += w[r];
+        const float target = a.topp * total;
+        unsigned used = 0u, keep = 0u;
+        float run = 0.0f;
+        for (int r = 0; r < k; r++) {
+            int best = -1;
+            for (int j = 0; j < k; j++)
+                if (!((used >> j) & 1u) && (best < 0 || w[j] > w[best])) best = j;
+            used |= 1u << best;
+            keep |= 1u << best;
+            run += w[best];
+            if (run >= target) break;
+        }
+        for (int r = 0; r < k; r++)
+            if (!((keep >> r) & 1u)) {
+                idx[r] = -1;
+                w[r] = 0.0f;
+            }
+    }
+    if (a.gap_out) {
+        float gap = (cand > k) ? (bk - rest) : INFINITY;
+        if (any_dropped) gap = fminf(gap, last_kept - best_dropped);
+        a.gap_out[t] = gap;
+    }
+}
+
 template <int MAXJ>  // candidate slots per lane: E <= 32 * MAXJ
 __device__ void select_core_j(const SelArgs &a, int64_t t, const float *s_sm, float *b_sm, int *pick) {
     const int lane = threadIdx.x & 31;
@@ -302,47 +346,7 @@ __device__ void select_core_j(const SelArgs &a, int64_t t, const float *s_sm, fl
         warp_argmax(rest, i);
     }
     const int cand = __popc(gmask) * gsz;
-
-    if (lane == 0) {
-        const int k = a.k;
-        int32_t *idx = a.idx_out + t * k;
-        float *w = a.w_out + t * k;
-        float sum = 0.0f;
-        for (int r = 0; r < k; r++)
-            if (pick[r] >= 0) sum += s_sm[pick[r]];
-        for (int r = 0; r < k; r++) {
-            idx[r] = pick[r];
-            w[r] = pick[r] >= 0 ? (s_sm[pick[r]] / sum) * a.rsf : 0.0f;
-        }
-        if (a.topp > 0.0f && a.topp < 1.0f) {
-            // rank the slots by weight (ties keep slot order), keep the shortest
-            // prefix that reaches topp * total
-            float total = 0.0f;
-            for (int r = 0; r < k; r++) total += w[r];
-            const float target = a.topp * total;
-            unsigned used = 0u, keep = 0u;
-            float run = 0.0f;
-            for (int r = 0; r < k; r++) {
-                int best = -1;
-                for (int j = 0; j < k; j++)
-                    if (!((used >> j) & 1u) && (best < 0 || w[j] > w[best])) best = j;
-                used |= 1u << best;
-                keep |= 1u << best;
-                run += w[best];
-                if (run >= target) break;
-            }
-            for (int r = 0; r < k; r++)
-                if (!((keep >> r) & 1u)) {
-                    idx[r] = -1;
-                    w[r] = 0.0f;
-                }
-        }
-        if (a.gap_out) {
-            float gap = (cand > k) ? (bk - rest) : INFINITY;
-            if (any_dropped) gap = fminf(gap, last_kept - best_dropped);
-            a.gap_out[t] = gap;
-        }
-    }
+    if (lane == 0) select_finish(a, t, s_sm, pick, bk, rest, last_kept, best_dropped, any_dropped, cand);
 }
 
 __device__ void select_core(const SelArgs &a, int64_t t, const float *s_sm, float *b_sm, int *pick) {
@@ -398,65 +402,65 @@ struct FusedRouteArgs {
     int32_t n_zero;
 };
 
-// Stable counting sort of P <= 32 * 2048 pairs by one block (sm: E + 48 ints).
-__device__ void bucket_small(const int32_t *idx, int P, int k, int E, int32_t *counts,
-                             int32_t *offsets, int32_t *list, int32_t *tok, int32_t *pos,
-                             int32_t *unique, int32_t *n_unique, uint32_t *flags, int *sm) {
-    int *cur = sm;
-    int *wt = sm + E;
-    const int tid = threadIdx.x, lane = tid & 31;
-    for (int e = tid; e < E; e += blockDim.x) cur[e] = 0;
-    __syncthreads();
+// Stable bucketing of a small batch (P = T * k <= 256 pairs) by one block:
+// every quantity is a direct count over the pairs (no scans over E).  The
+// same outputs as the counting sort: list sorted by (expert, pair), tok, pos
+// (-1 for dropped slots), counts, offsets [E+1], ascending unique experts.
+// sm: 2 * P ints.
+__device__ void bucket_tiny(const int32_t *idx, int P, int k, int E, int32_t *counts, int32_t *offsets,
+                            int32_t *list, int32_t *tok, int32_t *pos, int32_t *unique,
+                            int32_t *n_unique, uint32_t *flags, int *sm) {
+    int *pe = sm;         // [P] expert of each pair, -1 if dropped or invalid
+    int *first = sm + P;  // [P] pair is the first of its expert
+    const int tid = threadIdx.x;
     bool bad = false;
     for (int p = tid; p < P; p += blockDim.x) {
-        const int e = __ldcg(idx + p);
-        if (e >= E) bad = true;
-        else if (e >= 0) atomicAdd(&cur[e], 1);
+        int e = __ldcg(idx + p);
+        if (e >= E) {
+            bad = true;
+            e = -1;
+        }
+        pe[p] = e;
     }
     if (__syncthreads_or(bad) && tid == 0) raise_flag(flags, MOE_FLAG_BAD_EXPERT_INDEX);
-    const int per = (E + blockDim.x - 1) / blockDim.x;
-    const int e0 = tid * per, e1 = min(E, e0 + per);
-    int c = 0, nz = 0;
-    for (int e = e0; e < e1; e++) {
-        c += cur[e];
-        nz += cur[e] > 0;
-    }
-    int tot, nu;
-    const int off = block_exclusive_scan(c, wt, &tot);
-    const int uo = block_exclusive_scan(nz, wt, &nu);
-    int run = off, u = uo;
-    for (int e = e0; e < e1; e++) {
-        const int ce = cur[e];
-        counts[e] = ce;
-        offsets[e] = run;
-        if (ce > 0) unique[u++] = e;
-        cur[e] = run;
-        run += ce;
-    }
-    if (tid == 0) {
-        offsets[E] = tot;
-        *n_unique = nu;
+    for (int p = tid; p < P; p += blockDim.x) {
+        const int e = pe[p];
+        int f = e >= 0;
+        for (int j = 0; j < p && f; j++) f = pe[j] != e;
+        first[p] = f;
     }
     __syncthreads();
-    if (tid < 32) {
-        for (int base = 0; base < P; base += 32) {
-            const int p = base + lane;
-            const int e = p < P ? __ldcg(idx + p) : -1;
-            const bool valid = e >= 0 && e < E;
-            const unsigned mask = __match_any_sync(0xffffffffu, valid ? e : -1);
-            const int rank = __popc(mask & lanemask_lt());
-            const bool leader = (__ffs(mask) - 1) == lane;
-            int q = -1;
-            if (valid) q = cur[e] + rank;
-            __syncwarp();
-            if (valid) {
-                list[q] = p;
-                tok[q] = p / k;
-                if (leader) cur[e] += __popc(mask);
-            }
-            if (p < P) pos[p] = q;
-            __syncwarp();
+    for (int e = tid; e <= E; e += blockDim.x) {
+        int c = 0, lt = 0;
+        for (int j = 0; j < P; j++) {
+            const int ej = pe[j];
+            c += ej == e;
+            lt += ej >= 0 && ej < e;
         }
+        if (e < E) counts[e] = c;
+        offsets[e] = lt;
+    }
+    for (int p = tid; p < P; p += blockDim.x) {
+        const int e = pe[p];
+        if (e < 0) {
+            pos[p] = -1;
+            continue;
+        }
+        int q = 0, u = 0;
+        for (int j = 0; j < P; j++) {
+            const int ej = pe[j];
+            q += ej >= 0 && (ej < e || (ej == e && j < p));
+            u += first[j] && ej < e;
+        }
+        list[q] = p;
+        tok[q] = p / k;
+        pos[p] = q;
+        if (first[p]) unique[u] = e;
+    }
+    if (tid == 0) {
+        int nu = 0;
+        for (int j = 0; j < P; j++) nu += first[j];
+        *n_unique = nu;
     }
 }
 
@@ -496,8 +500,8 @@ __global__ void __launch_bounds__(RL_WARPS * 32) route_fused_small(FusedRouteArg
     for (int64_t t = wid; t < T; t += RL_WARPS)
         select_core(a.sel, t, s_all + t * E, b_all + t * E, picks + wid * 32);
     __syncthreads();
-    bucket_small(a.sel.idx_out, static_cast<int>(a.sel.T * a.sel.k), a.sel.k, E, a.counts, a.offsets,
-                 a.list, a.tok, a.pos, a.unique, a.n_unique, a.flags, reinterpret_cast<int *>(dsm));
+    bucket_tiny(a.sel.idx_out, static_cast<int>(a.sel.T * a.sel.k), a.sel.k, E, a.counts, a.offsets,
+                a.list, a.tok, a.pos, a.unique, a.n_unique, a.flags, reinterpret_cast<int *>(dsm));
     for (int i = threadIdx.x; i < a.n_zero; i += blockDim.x) a.zero_cnt[i] = 0;
     if (threadIdx.x == 0) *a.counter = 0u;
 }
@@ -581,7 +585,7 @@ moe_status launch_route_fused(const uint16_t *x, int64_t T, int64_t H, const flo
     a.n_zero = n_zero;
     const int E = cfg->n_experts;
     size_t smem = static_cast<size_t>(2 * T * E + RL_WARPS * 32) * sizeof(float);
-    const size_t bsm = static_cast<size_t>(E + 48) * sizeof(int);
+    const size_t bsm = static_cast<size_t>(2 * T * cfg->top_k) * sizeof(int);  // bucket_tiny
     if (bsm > smem) smem = bsm;
     if (smem > 48 * 1024 &&
         cudaFuncSetAttribute(route_fused_small, cudaFuncAttributeMaxDynamicSharedMemorySize,
