@@ -37,6 +37,35 @@ from int4_routed_expert_route_b200 import synthetic as syn  # noqa: E402
 METRIC = "MoE-layer tokens/s and int4 expert-weight HBM GB/s (fraction of roofline) on 1 B200"
 
 
+def source_sha256(files):
+    """sha256 over the named library sources (csrc/), in the order given."""
+    import hashlib
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, "int4_routed_expert_route_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def measured_traffic(kernel):
+    """DRAM bytes (read + write) per launch of `kernel` from the committed ncu
+    capture (profiles/roofline_traffic.txt), or None when the kernel's sources
+    changed after that capture (their sha256 no longer matches)."""
+    path = os.path.join(ROOT, "profiles", "roofline_traffic.txt")
+    if not os.path.exists(path):
+        return None
+    with open(path) as fh:
+        for line in fh:
+            f = line.split()
+            if not f or f[0].startswith("#") or f[0] != kernel:
+                continue
+            try:
+                return float(f[3]) if source_sha256(f[1].split(",")) == f[2] else None
+            except OSError:
+                return None
+    return None
+
+
 def measured_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -262,7 +291,8 @@ def run_ours(args, world, rank):
         achieved = float(np.mean(gu_bytes / (gu_ms * 1e-3))) / 1e9
         roof = {"kernel": kern, "bound": "hbm", "achieved": round(achieved, 1),
                 "peak": peaks["hbm_gbs"], "peak_source": peak_kind, "unit": "GB/s",
-                "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": None,
+                "frac": round(achieved / peaks["hbm_gbs"], 4),
+                "traffic": measured_traffic("gateup_decode") if T <= 8 else None,
                 "algorithmic_bytes_per_launch": int(np.mean(gu_bytes))}
         launches = 3 if T <= 8 else 6
     else:
@@ -272,8 +302,9 @@ def run_ours(args, world, rank):
         roof = {"kernel": kern, "bound": "tensor", "achieved": round(achieved, 1),
                 "peak": peaks["bf16_tflops"], "peak_source": peak_kind + " (bf16 burst)",
                 "unit": "TFLOP/s", "frac": round(achieved / peaks["bf16_tflops"], 4),
-                "traffic": None, "algorithmic_flops_per_launch": float(np.mean(gu_flops))}
-        launches = 5
+                "traffic": measured_traffic("tc_ffn<1>"),
+                "algorithmic_flops_per_launch": float(np.mean(gu_flops))}
+        launches = 7  # router logits, select, bucket, gather, two tc_ffn passes, combine
     total_flops_step = (pairs + T) * 2.0 * 3 * I * H
     res = {
         "metric": METRIC,
