@@ -154,41 +154,49 @@ __device__ __forceinline__ bool bfly_writer(int lane) {
 // 2^-e as an exact fp32 constant (0 <= e <= 20).
 __device__ __forceinline__ float exp2_neg(int e) { return __uint_as_float(static_cast<uint32_t>(127 - e) << 23); }
 
-// Loads a lane's activation slice (bf16 or fp32 source) pre-scaled by 2^-e.
-// f2 index w*PW + p = (column w*CPW + 2p, column w*CPW + 2p + 1), each
-// scaled by 2^-e of its code position.
-template <int BITS, typename Src>
-__device__ __forceinline__ float act_at(const Src *src, int col);
-template <>
-__device__ __forceinline__ float act_at<4, uint16_t>(const uint16_t *src, int col) { return bf16_bits_to_float(src[col]); }
-template <>
-__device__ __forceinline__ float act_at<8, uint16_t>(const uint16_t *src, int col) { return bf16_bits_to_float(src[col]); }
-template <>
-__device__ __forceinline__ float act_at<2, uint16_t>(const uint16_t *src, int col) { return bf16_bits_to_float(src[col]); }
-template <>
-__device__ __forceinline__ float act_at<4, float>(const float *src, int col) { return src[col]; }
-template <>
-__device__ __forceinline__ float act_at<8, float>(const float *src, int col) { return src[col]; }
-template <>
-__device__ __forceinline__ float act_at<2, float>(const float *src, int col) { return src[col]; }
-
+// Loads a lane's NC activations (contiguous, 16-byte aligned: the chunk's
+// column offset is a multiple of NC) with 16-byte vector loads — every lane of
+// every block reads them at the same moment, so scalar loads would queue up in
+// L2 — and pre-scales them by 2^-e of their code position: f2 index w*PW + p
+// holds (column w*CPW + 2p, column w*CPW + 2p + 1).
 template <int BITS, typename Src>
 __device__ __forceinline__ void load_act(const Src *src, bool have, f2 *out) {
     using D = Dec<BITS>;
-    constexpr int CW = Chunk<BITS>::W, PW = D::CPW / 2;
-    {
+    constexpr int CW = Chunk<BITS>::W, PW = D::CPW / 2, NC = CW * D::CPW;
+    float v[NC];
 #pragma unroll
-        for (int w = 0; w < CW; w++)
+    for (int i = 0; i < NC; i++) v[i] = 0.0f;
+    if (have) {
+        if constexpr (sizeof(Src) == 2) {
+            static_assert(NC % 8 == 0, "bf16 activations come in 16-byte groups of 8");
 #pragma unroll
-            for (int p = 0; p < PW; p++) {
-                float v0 = 0.f, v1 = 0.f;
-                if (have) {
-                    v0 = act_at<BITS, Src>(src, w * D::CPW + 2 * p) * exp2_neg(D::exp_of(2 * p));
-                    v1 = act_at<BITS, Src>(src, w * D::CPW + 2 * p + 1) * exp2_neg(D::exp_of(2 * p + 1));
+            for (int i = 0; i < NC / 8; i++) {
+                const uint4 q = *reinterpret_cast<const uint4 *>(src + 8 * i);
+                const uint32_t w4[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+                for (int j = 0; j < 4; j++) {
+                    v[8 * i + 2 * j] = __uint_as_float(w4[j] << 16);
+                    v[8 * i + 2 * j + 1] = __uint_as_float(w4[j] & 0xffff0000u);
                 }
-                out[w * PW + p] = f2_make(v0, v1);
             }
+        } else {
+            static_assert(NC % 4 == 0, "fp32 activations come in 16-byte groups of 4");
+#pragma unroll
+            for (int i = 0; i < NC / 4; i++) {
+                const float4 q = *reinterpret_cast<const float4 *>(src + 4 * i);
+                v[4 * i] = q.x;
+                v[4 * i + 1] = q.y;
+                v[4 * i + 2] = q.z;
+                v[4 * i + 3] = q.w;
+            }
+        }
     }
+#pragma unroll
+    for (int w = 0; w < CW; w++)
+#pragma unroll
+        for (int p = 0; p < PW; p++)
+            out[w * PW + p] = f2_make(v[w * D::CPW + 2 * p] * exp2_neg(D::exp_of(2 * p)),
+                                      v[w * D::CPW + 2 * p + 1] * exp2_neg(D::exp_of(2 * p + 1)));
 }
 
 // acc += decoded(chunk) . act  for one lane chunk.
