@@ -84,6 +84,10 @@ __device__ __forceinline__ DSeg dec_seg(const DecodeArgs &a, int64_t s) {
 // contiguous ranges.
 __device__ __forceinline__ void dec_block_rows(int64_t nseg, int64_t seg_rows, int64_t &r0, int64_t &r1) {
     const int64_t nb = gridDim.x, b = blockIdx.x;
+    if (nseg <= 0) {
+        r0 = r1 = 0;
+        return;
+    }
     if (nseg <= nb) {
         const int64_t bps = nb / nseg;
         const int64_t s = b / bps, piece = b % bps;
@@ -384,7 +388,7 @@ constexpr int DN_TILE = 64;
 constexpr int kMaxTiles = 768;  // counters live in the 4 KiB workspace header
 
 template <int BITS, int TG, int U>
-__global__ void __launch_bounds__(384, 1) down_decode(DecodeArgs a) {
+__global__ void __launch_bounds__(TG == 1 ? 512 : 384, 1) down_decode(DecodeArgs a) {
     using D = Dec<BITS>;
     constexpr int CW = Chunk<BITS>::W;
     constexpr int NP = CW * (D::CPW / 2);
@@ -544,7 +548,7 @@ static int dec_sm_count() {
     return n;
 }
 
-static constexpr int GU_U = 8, DN_U = 8;  // rows per ring stage
+static constexpr int GU_U = 8, DN_U = 4;  // rows per ring stage
 
 bool decode_ok(int64_t T, int64_t H, int64_t I, int32_t k, int32_t bits) {
     (void)k;
@@ -578,7 +582,8 @@ static moe_status launch_decode_bits(DecodeArgs a, cudaStream_t stream, cudaEven
     {
         DecodeArgs d = a;
         d.kw = kw_dn;
-        d.rg = 12 / kw_dn > 0 ? 12 / kw_dn : 1;
+        const int dn_warps = TG == 1 ? 16 : 12;  // 16 warps at T = 1 (128 registers suffice there)
+        d.rg = dn_warps / kw_dn > 0 ? dn_warps / kw_dn : 1;
         const int threads = 32 * d.kw * d.rg;
         const size_t smem = static_cast<size_t>(DN_RMAX) * TG * d.kw * sizeof(float) +
                             static_cast<size_t>(threads / 32) * DN_S * DN_U * 32 * D::CH;
