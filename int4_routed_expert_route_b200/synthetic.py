@@ -8,7 +8,7 @@ Distributions (the workload statement of the layer):
   expert weights  W ~ N(0, 0.02) fp32, one seed per (config, layer, expert, matrix)
   router gate     G [E, H] ~ N(0, 0.02) fp32
   router bias     U(-a, a), or Zipf(s=1.1) over a seeded random expert ranking,
-                  bias_e = 0.5 * rank_e^-1.1 (magnitude 0.5 is this build's choice)
+                  bias_e = 0.5 * rank_e^-1.1 (the magnitude 0.5 is a chosen value; none is given)
   activations     x ~ N(0, 1) rounded to bf16, one seed per call
 """
 from dataclasses import dataclass, field, replace
