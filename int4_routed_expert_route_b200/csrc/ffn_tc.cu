@@ -133,7 +133,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
     return false;
 }
 
-// Warp-wide bounded wait: lane 0 polls, the other lanes take its result.
+// Warp-wide bounded wait: lane 0 polls, the other lanes take its verdict.
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, int lane) {
     bool ok = true;
     if (lane == 0) ok = mbar_wait(bar, parity);
