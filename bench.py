@@ -47,11 +47,11 @@ def source_sha256(files):
     return h.hexdigest()
 
 
-def measured_traffic(kernel):
+def measured_traffic(kernel, path=None):
     """DRAM bytes (read + write) per launch of `kernel` from the committed ncu
     capture (profiles/roofline_traffic.txt), or None when the kernel's sources
     changed after that capture (their sha256 no longer matches)."""
-    path = os.path.join(ROOT, "profiles", "roofline_traffic.txt")
+    path = path or os.path.join(ROOT, "profiles", "roofline_traffic.txt")
     if not os.path.exists(path):
         return None
     with open(path) as fh:
