@@ -97,3 +97,40 @@ def test_library_has_no_unresolved_internal_symbols(so):
     from int4_routed_expert_route_b200 import build
     out = subprocess.run(["nm", "-u", build.LIB], capture_output=True, text=True).stdout
     assert "_ZN3moe" not in out
+
+
+def test_host_side_path_and_size_contracts(so):
+    """Refusals the boundary makes on the host, before any launch (no GPU needed)."""
+    import int4_routed_expert_route_b200 as m
+    L = m.load()
+    fake = ctypes.c_void_p(0x1000)
+    cfg = m.router_cfg(256, 8, 8, 4, 2.5)
+    big = 1 << 40
+
+    def fwd(T, H, I, bits, path, ws_bytes=big):
+        return L.moe_layer_forward_ex(fake, T, H, I, fake, fake, ctypes.byref(cfg), fake, None,
+                                      bits, fake, None, None, fake, ws_bytes, path, 0, None, None)
+
+    # the tensor-core path takes int4 experts with H, I multiples of 128 only
+    assert fwd(256, 6144, 2048, 8, m.PATH_TENSOR) == 2
+    assert fwd(256, 6144 + 64, 2048, 4, m.PATH_TENSOR) == 2
+    # the CUDA-core path stops at 4096 tokens
+    assert fwd(4097, 6144, 2048, 4, m.PATH_GEMV) == 2
+    # an empty batch is fine and launches nothing
+    assert fwd(0, 6144, 2048, 4, m.PATH_AUTO) == 0
+    # AUTO runs int8/int2 layers on the CUDA-core path: its workspace must fit in the one
+    # sized for AUTO (which plans the tensor path from 64 tokens on)
+    for T in (1, 8, 63, 64, 256, 4096):
+        auto = m.moe_layer_workspace_bytes(T, 6144, 2048, cfg)
+        gemv = m.moe_layer_workspace_bytes(T, 6144, 2048, cfg, m.PATH_GEMV)
+        assert 0 < gemv <= auto, T
+        assert fwd(T, 6144, 2048, 8, m.PATH_AUTO, ws_bytes=gemv - 1) == 4  # sized for GEMV
+    # stack and RMSNorm argument errors
+    assert L.moe_stack_forward(fake, 1, 6144, 2048, -1, None, ctypes.byref(cfg), 1e-6, None, None,
+                               fake, big, None) == 1
+    need = L.moe_stack_workspace_bytes(1, 6144, 2048, ctypes.byref(cfg))
+    assert need > m.moe_layer_workspace_bytes(1, 6144, 2048, cfg)
+    assert L.moe_stack_forward(fake, 1, 6144, 2048, 0, None, ctypes.byref(cfg), 1e-6, None, None,
+                               fake, need - 1, None) == 4
+    assert L.moe_rmsnorm_bf16(fake, 1, 6144, ctypes.c_float(-1.0), fake, None) == 1
+    assert L.moe_rmsnorm_bf16(fake, 1, 6144, ctypes.c_float(float("nan")), fake, None) == 1
