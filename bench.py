@@ -37,13 +37,22 @@ from int4_routed_expert_route_b200 import synthetic as syn  # noqa: E402
 METRIC = "MoE-layer tokens/s and int4 expert-weight HBM GB/s (fraction of roofline) on 1 B200"
 
 
+def _code_only(text):
+    """Source text without comments, whitespace collapsed: what the compiler sees."""
+    import re
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    return " ".join(text.split())
+
+
 def source_sha256(files):
-    """sha256 over the named library sources (csrc/), in the order given."""
+    """sha256 over the code (comments and layout ignored) of the named library
+    sources (csrc/), in the order given."""
     import hashlib
     h = hashlib.sha256()
     for f in files:
-        with open(os.path.join(ROOT, "int4_routed_expert_route_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, "int4_routed_expert_route_b200", "csrc", f)) as fh:
+            h.update(_code_only(fh.read()).encode())
     return h.hexdigest()
 
 

@@ -3,12 +3,13 @@
 // Batch-union grouped GEMM ("Show HN: running GLM 5.2 on a slow computer",
 // implemented features: batch-union MoE, each unique expert read once and
 // applied to all positions routed to it; dequant-on-use int4 weights).  Two
-// passes, each a persistent kernel over tiles of 128 weight rows x <=256 tokens
+// passes, each a persistent kernel over tiles of 128 weight rows x <=192 tokens
 // of one expert:
 //   pass 1 (gate/up): D_g = Q_g X^T, D_u = Q_u X^T  (bf16 x bf16 -> fp32 in TMEM)
 //                     h = silu(s_g D_g) * (s_u D_u)  -> fp16 h[pair][I]
 //   pass 2 (down):    D = Q_d H^T                   (fp16 x fp16 -> fp32 in TMEM)
-//                     y[t] += w_pair * s_d * D      (red.add into fp32 y)
+//                     yp[pair] = s_d * D            (fp32 per-pair partials; the
+//                     combine kernel adds them per token in slot order)
 // int4 codes are exact in bf16 and fp16, so dequantising to 16 bits adds no
 // error; the row scale is applied in the epilogue in fp32.
 //
