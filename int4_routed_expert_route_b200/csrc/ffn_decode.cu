@@ -3,19 +3,26 @@
 // Bandwidth design for HBM-bound int4 GEMV ("Show HN: running GLM 5.2 on a slow
 // computer", implemented features: dequant-on-use, batch-union MoE; here the
 // experts are resident in HBM instead of being streamed from disk):
-//  - Gate/up: the rows of all unique experts of the batch (shared expert first)
-//    form one row space; each block takes an equal contiguous range of it, so
-//    every SM streams the same number of bytes.  Warp (kw, rg) owns the 16-byte
-//    chunks [32kw, 32kw+32) of the rows rg, rg+RG, ... of the range; its slice of
-//    the activations stays in registers.  Each lane keeps two sets of U rows of
-//    128-bit streaming loads in flight (register double buffering).
+//  - The rows of all unique experts of the batch (shared expert first) form one
+//    row space; blocks split it so that each works inside one expert (blocks
+//    per expert = grid / experts), every SM streaming about the same bytes.
+//    Warp (kw, rg) owns the 16-byte chunks [32kw, 32kw+32) of the rows
+//    rg, rg+RG, ... of its range; its activation slice (pre-scaled by 2^-e,
+//    read with 16-byte loads) stays in registers.  Each lane streams its own
+//    chunks through a private cp.async ring in shared memory.
+//  - An int4 code c at bit 4p of a word is decoded as the exact float
+//    2^23 + c*2^e (one lop3 with 0x4B000000), one packed subtract and one packed
+//    FMA per pair of codes.
 //  - Partial dot products are reduced across the warp with a reduce-scatter
 //    butterfly (V values in V-1 + log2(32/V) shuffles instead of 5V) and across
 //    the K-slice warps once per run in shared memory, in a fixed order.
-//  - Down: each block owns a contiguous range of output rows of H and loops
-//    over every unique expert of the batch, so it can apply the routing weights
-//    and the shared expert itself and write y once: the weighted combine is
-//    fused and deterministic (no atomics, no extra launch).
+//  - Down: blocks write per-pair partials and count the finished rows of every
+//    64-row tile of H; the block that completes a tile adds each token's
+//    partials in slot order and writes y once: the weighted combine is fused
+//    and deterministic (no atomics on y, no extra launch).
+//  - The gate/up and down kernels launch with programmatic stream
+//    serialization: each waits for its predecessor only where it reads that
+//    kernel's output (down issues its weight prologue before waiting for h).
 #include <cstring>
 
 #include "common.cuh"
