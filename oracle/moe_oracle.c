@@ -30,6 +30,12 @@
  *    weights w_i = (s_i / sum_i s_i) * rsf in fp32 with the sum in slot order.
  * Readings where the pages are silent are listed in the design notes and in the
  * comments below.
+ *
+ * Parity unpinned: the expert top-p step (route_one) follows a reading of an
+ * option the pages name ("--topp 0.7") without defining it -- rank the slots by
+ * weight, keep the shortest prefix reaching topp * total, drop the rest without
+ * renormalising.  Its golden cases are written from that reading, so nothing
+ * outside the reading pins it.
  */
 #include <math.h>
 #include <stdint.h>
