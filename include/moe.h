@@ -263,6 +263,11 @@ MOE_API moe_status moe_layer_forward(const uint16_t *x, int64_t T, int64_t H, in
  *   events  HOST array of MOE_LAYER_EVENTS events, nullable: event i is recorded
  *           on `stream` before stage i (0 router, 1 bucket, 2 gate/up, 3 down,
  *           4 combine) and event 5 after the last stage, for per-stage timing.
+ *           Null entries are skipped.  On the decode path the kernels overlap
+ *           their start-up with their predecessor (programmatic dependent
+ *           launch); an event recorded between two of them serialises them, so
+ *           to time a whole call pass only events 0 and 5.  Inside a stream
+ *           capture the events are recorded as external event nodes.
  *   accumulate  0: y is overwritten; 1: y += layer output (residual add).
  */
 #define MOE_LAYER_EVENTS 6
