@@ -344,7 +344,10 @@ def run_ours(args, world, rank):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "int4 weights, fp32 accumulate (bf16 activations)",
+        "dtype": "f32" if T < 64 else "bf16",
+        "dtype_detail": ("int4 codes decoded to f32, f32 FMA (CUDA cores)" if T < 64 else
+                         "int4 codes converted to bf16 (gate/up) / f16 (down), tcgen05 MMA "
+                         "with f32 accumulation") + "; bf16 activations",
         "data": "synthetic (seeded N(0,0.02) weights quantised on device; x ~ N(0,1) bf16)",
         "config": {"workload": workload_name(cfg), "tokens_per_step": T,
                    "l2": "flushed before every step (256 MB write, outside the timed events)",
@@ -454,7 +457,8 @@ def run_stack(args, world, rank):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": f"int{cfg.bits} weights, fp32 accumulate (bf16 activations, fp32 residual)",
+        "dtype": "f32",
+        "dtype_detail": f"int{cfg.bits} codes decoded to f32, f32 FMA; bf16 layer inputs, f32 residual",
         "data": "synthetic (seeded N(0,0.02) weights quantised on device; residual ~ N(0,1) fp32)",
         "config": {"workload": f"{cfg.name}: {nl} layers, T={T} per step, H={H} I={I} E={cfg.E}+1 "
                                f"shared top-{cfg.k}, RMSNorm eps 1e-6 + fp32 residual",
