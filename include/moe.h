@@ -104,6 +104,9 @@ typedef struct moe_router_cfg {
 } moe_router_cfg;
 
 /* ------------------------------------------------------------------------- */
+/* Library plumbing below (status names, version, workspace header): the pages
+ * have no counterpart; these exist because the library never allocates and
+ * reports device-side problems through the caller's workspace. */
 
 /* Human-readable status name (static storage). */
 MOE_API const char *moe_status_str(moe_status s);
@@ -283,6 +286,12 @@ MOE_API moe_status moe_layer_forward_ex(const uint16_t *x, int64_t T, int64_t H,
  * RMSNorm without weight, rounded to bf16 (the layer input of a stack):
  *   out[t,j] = bf16( v[t,j] / sqrt(mean_j v[t,j]^2 + eps) ), fp32 arithmetic.
  *   v [T, H] fp32;  out [T, H] bf16
+ * Source: the pages run a token through 75 consecutive MoE layers ("Enthusiast
+ * ran GLM-5.2 on a laptop with 25 GB of RAM"; "Show HN", "disk-streaming MoE
+ * execution"); the norm between them is the model's pre-layer RMSNorm, taken
+ * here without its learned weight (unit gamma) since no weights are loaded.
+ * Errors: MOE_ERR_INVALID_ARG for T < 0, H <= 0, null pointers with T > 0, or
+ * eps negative / NaN; no workspace.
  */
 MOE_API moe_status moe_rmsnorm_bf16(const float *v, int64_t T, int64_t H, float eps, uint16_t *out,
                             cudaStream_t stream);
