@@ -193,6 +193,8 @@ WORKLOADS = {
     "decode": syn.DECODE,
     "prefill": syn.PREFILL,
     "small_batch": syn.SMALL_BATCH.with_(T=32),
+    # adaptive expert top-p 0.7: slots beyond the cumulative weight are dropped
+    "decode_topp": syn.DECODE.with_(name="glm-scale decode, expert top-p 0.7", topp=0.7),
     # MTP verify: 4 drafts from one position, x_t = x_0 + 0.05 n_t, Zipf router
     "mtp_verify": syn.SMALL_BATCH.with_(name="glm-scale MTP verify, 4 correlated drafts, zipf bias", T=4),
 }
