@@ -31,11 +31,13 @@
  * Readings where the pages are silent are listed in the design notes and in the
  * comments below.
  *
- * Parity unpinned: the expert top-p step (route_one) follows a reading of an
- * option the pages name ("--topp 0.7") without defining it -- rank the slots by
- * weight, keep the shortest prefix reaching topp * total, drop the rest without
- * renormalising.  Its golden cases are written from that reading, so nothing
- * outside the reading pins it.
+ * The expert top-p step (route_one) follows a reading of an option the pages
+ * name ("--topp 0.7") without defining it: rank the slots by weight, keep the
+ * shortest prefix reaching topp * total, drop the rest without renormalising.
+ * That reading is pinned by properties checked on random weight vectors (the
+ * kept slots are a prefix of the weight order, their sum reaches the target, a
+ * prefix one slot shorter does not, kept weights are unchanged, dropped slots
+ * read -1 / 0) and by hand-worked golden cases; the rule itself stays a reading.
  */
 #include <math.h>
 #include <stdint.h>

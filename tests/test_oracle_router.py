@@ -167,3 +167,88 @@ def test_bad_router_configs_rejected(orc):
     for k, ng, tkg in [(9, 1, 1), (2, 3, 1), (5, 4, 2), (1, 8, 1), (2, 2, 3)]:
         with pytest.raises(orc.OracleError):
             orc.route_from_scores(s, z, k, ng, tkg)
+
+
+# Sigmoid closed forms.  For r > 0, sigmoid(ln r) = r / (1 + r).  The logits below
+# are exact fp32 values (fp32(ln r), or 0, or 20) and the fp32 rounding of the
+# true sigmoid of each is the rational r/(1+r) (resp. 1/2, 1): the distance of
+# sigmoid(fp32(ln r)) from r/(1+r) is at most 0.11 ulp of the result below the
+# rounding boundary, derived from |fp32(ln r) - ln r| <= 2^-24 * |ln r| and
+# sigmoid' = s(1 - s).  sigmoid(20) = 1 - 2.06e-9 lies within 2^-25 of 1.
+SIGMOID_PINS = [
+    ("0x0p+0", 0.5),
+    ("0x1.193ea8p+0", 0.75),     # fp32(ln 3)
+    ("-0x1.193ea8p+0", 0.25),    # fp32(-ln 3)
+    ("0x1.f2272ap+0", 0.875),    # fp32(ln 7)
+    ("-0x1.f2272ap+0", 0.125),   # fp32(-ln 7)
+    ("0x1.5aa164p+1", 0.9375),   # fp32(ln 15)
+    ("0x1.4p+4", 1.0),           # 20
+]
+
+
+def test_scores_closed_form_sigmoid(orc):
+    """Token scores against closed forms, with the logit formed three ways so
+    that a transposed gate matrix, a dropped product or a wrong operand shows:
+    token 0 is one-hot 1.0 at column 3 (logit = G[e,3]); token 1 is 2.0 at column
+    10 with G[e,10] = logit/2; token 2 is 1.0 at column 20 and 2.0 at column 41
+    with G[e,20] = logit/2 and G[e,41] = logit/4 (all exact in fp32)."""
+    E, H = len(SIGMOID_PINS), 64
+    t_of = np.array([float.fromhex(h) for h, _ in SIGMOID_PINS], np.float32)
+    want = np.array([v for _, v in SIGMOID_PINS], np.float32)
+    G = np.zeros((E, H), np.float32)
+    G[:, 3] = t_of
+    G[:, 10] = t_of / np.float32(2)
+    G[:, 20] = t_of / np.float32(2)
+    G[:, 41] = t_of / np.float32(4)
+    x = np.zeros((3, H), np.float32)
+    x[0, 3] = 1.0
+    x[1, 10] = 2.0
+    x[2, 20] = 1.0
+    x[2, 41] = 2.0
+    xb = orc.f32_to_bf16_bits(x)
+    # the rows of G other than those columns are zero, so every expert's logit is t_of[e]
+    r = orc.route(xb, G, np.zeros(E, np.float32), k=1)
+    for t in range(3):
+        assert np.array_equal(r["scores"][t], want), (t, r["scores"][t], want)
+    # one row of G per expert: moving expert e's pin to another row moves its score
+    r2 = orc.route(xb, G[::-1].copy(), np.zeros(E, np.float32), k=1)
+    assert np.array_equal(r2["scores"][0], want[::-1])
+
+
+def test_expert_topp_properties(orc):
+    """Expert top-p (the reading of the "--topp" option in "Show HN: running GLM
+    5.2 on a slow computer", option list and community benchmarks): on random
+    weight vectors the kept slots are the shortest prefix of the slots ranked by
+    weight (ties to the lower slot) whose fp32 running sum reaches topp * total;
+    kept slots keep their expert and weight (no renormalisation); dropped slots
+    read index -1 and weight 0."""
+    rng = np.random.default_rng(11)
+    n, E = 600, 16
+    for k in (2, 5, 8):
+        s = rng.uniform(0.01, 0.99, (n, E)).astype(np.float32)
+        s[::5] = np.round(s[::5] * 4) / 4  # coarse scores: equal weights
+        bias = np.zeros(E, np.float32)
+        full = orc.route_from_scores(s, bias, k, 1, 1, 2.5)
+        for topp in (0.1, 0.3, 0.5, 0.7, 0.9, 0.99):
+            r = orc.route_from_scores(s, bias, k, 1, 1, 2.5, topp=topp)
+            for t in range(n):
+                w, idx = full["w"][t], full["idx"][t]
+                kept = r["idx"][t] >= 0
+                m = int(kept.sum())
+                assert m >= 1
+                assert np.array_equal(r["idx"][t][kept], idx[kept])
+                assert np.array_equal(r["w"][t][kept], w[kept])
+                assert np.all(r["idx"][t][~kept] == -1) and np.all(r["w"][t][~kept] == 0)
+                order = sorted(range(k), key=lambda i: (-float(w[i]), i))
+                assert set(np.nonzero(kept)[0].tolist()) == set(order[:m]), (t, topp, w)
+                total = np.float32(0)
+                for i in range(k):
+                    total = np.float32(total + w[i])
+                target = np.float32(np.float32(topp) * total)
+                run = np.float32(0)
+                runs = []
+                for i in order:
+                    run = np.float32(run + w[i])
+                    runs.append(run)
+                assert runs[m - 1] >= target
+                assert m == 1 or runs[m - 2] < target
