@@ -30,6 +30,7 @@ def lib():
         path = _build.build()
         L = ctypes.CDLL(path)
         L.orc_num_threads.restype = ctypes.c_int
+        L.orc_set_num_threads.argtypes = [ctypes.c_int]
         L.orc_row_bytes.restype = _i64
         L.orc_row_bytes.argtypes = [ctypes.c_int, _i64]
         L.orc_double_to_bf16.restype = ctypes.c_uint16
@@ -74,6 +75,11 @@ def _ok(rc, what):
 
 def num_threads() -> int:
     return lib().orc_num_threads()
+
+
+def set_num_threads(n: int) -> None:
+    """Threads the expert FFN rows are split over (results do not depend on it)."""
+    lib().orc_set_num_threads(int(n))
 
 
 def row_bytes(bits: int, cols: int) -> int:

@@ -1,9 +1,9 @@
 """Compile the plain-C oracle into oracle/liboracle.so (test infrastructure only).
 
 Flags keep the C semantics the oracle is written for: no fast-math, no FMA
-contraction, IEEE float division.  OpenMP only splits independent tokens / rows
-across threads; every output element is still computed by one thread in the
-order written in the source.
+contraction, IEEE float division.  OpenMP only splits independent rows (of a
+quantised matrix, of an expert FFN's outputs) across threads; every output
+element is still computed by one thread in the order written in the source.
 """
 import os
 import subprocess

@@ -60,6 +60,17 @@ int orc_num_threads(void)
 #endif
 }
 
+/* Threads the expert FFN rows are split over (1 = serial).  Every output value
+ * is computed by one thread in the order written here, whatever the count. */
+void orc_set_num_threads(int n)
+{
+#ifdef _OPENMP
+    if (n > 0) omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+}
+
 /* ------------------------------------------------------------------ */
 /* bf16 helpers                                                        */
 /* ------------------------------------------------------------------ */
@@ -378,7 +389,6 @@ int orc_route(const uint16_t *x, int64_t T, int64_t H, const float *G, const flo
 {
     if (check_router_cfg(E, k, n_group, topk_group)) return ORC_EINVAL;
     int err = 0;
-#pragma omp parallel for schedule(dynamic)
     for (int64_t t = 0; t < T; t++) {
         float *s = (float *)malloc(sizeof(float) * (size_t)E);
         double gap, ggap;
@@ -460,6 +470,8 @@ static void ffn_token(const orc_expert *ex, const double *x, int64_t H, int64_t 
                       double *y)
 {
     int64_t rbh = orc_row_bytes(ex->bits, H), rbi = orc_row_bytes(ex->bits, I);
+    /* rows are independent: each is computed by one thread */
+#pragma omp parallel for schedule(static)
     for (int64_t i = 0; i < I; i++) {
         double g = 0.0, u = 0.0;
         const uint8_t *rg = ex->qg + i * rbh, *ru = ex->qu + i * rbh;
@@ -469,6 +481,7 @@ static void ffn_token(const orc_expert *ex, const double *x, int64_t H, int64_t 
         }
         h[i] = silu(g) * u;
     }
+#pragma omp parallel for schedule(static)
     for (int64_t j = 0; j < H; j++) {
         double acc = 0.0;
         const uint8_t *rd = ex->qd + j * rbi;
@@ -484,7 +497,6 @@ int orc_expert_ffn(const uint16_t *x, int64_t T, int64_t H, int64_t I, const uin
     orc_expert ex = {qg, sg, qu, su, qd, sd, bits};
     float d; int lo, hi;
     if (qrange(bits, &d, &lo, &hi)) return ORC_EINVAL;
-#pragma omp parallel for schedule(dynamic)
     for (int64_t t = 0; t < T; t++) {
         double *xd = (double *)malloc(sizeof(double) * (size_t)H);
         double *h = (double *)malloc(sizeof(double) * (size_t)I);
@@ -525,7 +537,6 @@ int orc_layer(const uint16_t *x, int64_t T, int64_t H, int64_t I, const float *G
         if (e >= 0 && (!qg[e] || !sg[e] || !qu[e] || !su[e] || !qd[e] || !sd[e])) return ORC_EMISSING;
     }
     int err = 0;
-#pragma omp parallel for schedule(dynamic)
     for (int64_t t = 0; t < T; t++) {
         double *xd = (double *)malloc(sizeof(double) * (size_t)H);
         double *h = (double *)malloc(sizeof(double) * (size_t)I);
