@@ -178,8 +178,10 @@ MOE_API moe_status moe_route_topk(const uint16_t *x, int64_t T, int64_t H, const
  * minus 256, exceeds it returns MOE_ERR_WORKSPACE before anything is launched
  * (the scratch is T * n_experts fp32 logits: up to T = 4096 with 256 experts).
  * The first call on a device looks up the array's address (make it before any
- * stream capture).  All calls share the array: calls that overlap on the GPU race
- * and must be serialised by the caller.  Allocates nothing.
+ * stream capture); only a successful lookup is kept, so a call whose lookup
+ * failed returns MOE_ERR_CUDA and the next call tries again.  All calls share
+ * the array: calls that overlap on the GPU race and must be serialised by the
+ * caller.  Allocates nothing.
  */
 MOE_API size_t moe_route_noalloc_max_scratch_bytes(void);
 MOE_API moe_status moe_route_topk_noalloc(const uint16_t *x, int64_t T, int64_t H,
@@ -284,7 +286,8 @@ MOE_API moe_status moe_layer_forward_ex(const uint16_t *x, int64_t T, int64_t H,
 
 /*
  * RMSNorm without weight, rounded to bf16 (the layer input of a stack):
- *   out[t,j] = bf16( v[t,j] / sqrt(mean_j v[t,j]^2 + eps) ), fp32 arithmetic.
+ *   out[t,j] = bf16( v[t,j] * r[t] ),  r[t] = 1 / sqrt(mean_j v[t,j]^2 + eps),
+ *   fp32 arithmetic with IEEE square root and division, nearest-even bf16.
  *   v [T, H] fp32;  out [T, H] bf16
  * Source: the pages run a token through 75 consecutive MoE layers ("Enthusiast
  * ran GLM-5.2 on a laptop with 25 GB of RAM"; "Show HN", "disk-streaming MoE

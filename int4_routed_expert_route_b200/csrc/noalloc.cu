@@ -10,9 +10,11 @@
 // logits) from a file-scope device array that lives in the library image.
 //
 // The array holds kRouteScratchBytes (4 MiB) on every GPU that loads the library,
-// until the process exits.  Its device address is looked up once per device with
-// cudaGetSymbolAddress on the first call made while that device is current; that
-// first call should therefore happen before any stream capture.  All calls share
+// until the process exits.  Its device address is looked up with
+// cudaGetSymbolAddress by the first call made while that device is current, and
+// kept once the lookup succeeds; a failed lookup returns MOE_ERR_CUDA and is
+// tried again by the next call.  That first call should happen before any stream
+// capture.  All calls share
 // the array, so calls whose kernels overlap on the GPU (different streams, or
 // different host threads) race on it and must be serialised by the caller.  The
 // router overwrites every scratch element it reads, so nothing needs clearing.
@@ -33,9 +35,23 @@ constexpr size_t kRouteScratchBytes = static_cast<size_t>(4) << 20;
 static __device__ __align__(256) unsigned char g_route_scratch[kRouteScratchBytes];
 
 constexpr int kMaxDevices = 64;
-static std::once_flag g_scratch_once[kMaxDevices];
-static void *g_scratch_ptr[kMaxDevices];
-static cudaError_t g_scratch_err[kMaxDevices];
+static std::mutex g_scratch_mu[kMaxDevices];
+static void *g_scratch_ptr[kMaxDevices];  // set once a lookup has succeeded
+
+// Device address of the scratch array on the current device `dev`, looked up
+// on first use; only a successful lookup is cached.
+static void *scratch_address(int dev) {
+    std::lock_guard<std::mutex> lock(g_scratch_mu[dev]);
+    if (g_scratch_ptr[dev] == nullptr) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_route_scratch) != cudaSuccess) {
+            cudaGetLastError();  // the failure is reported through the status, not left pending
+            return nullptr;
+        }
+        g_scratch_ptr[dev] = p;
+    }
+    return g_scratch_ptr[dev];
+}
 
 static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -60,12 +76,8 @@ extern "C" MOE_API moe_status moe_route_topk_noalloc(const uint16_t *x, int64_t 
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
     if (dev < 0 || dev >= kMaxDevices) return MOE_ERR_UNSUPPORTED;
-    std::call_once(g_scratch_once[dev], [dev]() {
-        void *p = nullptr;
-        g_scratch_err[dev] = cudaGetSymbolAddress(&p, g_route_scratch);
-        g_scratch_ptr[dev] = p;
-    });
-    if (g_scratch_err[dev] != cudaSuccess || g_scratch_ptr[dev] == nullptr) return MOE_ERR_CUDA;
-    return launch_route(x, T, H, gate, bias, cfg, idx_out, w_out, gap_out,
-                        static_cast<double *>(g_scratch_ptr[dev]), stream);
+    void *scratch = scratch_address(dev);
+    if (scratch == nullptr) return MOE_ERR_CUDA;
+    return launch_route(x, T, H, gate, bias, cfg, idx_out, w_out, gap_out, static_cast<double *>(scratch),
+                        stream);
 }

@@ -1,6 +1,7 @@
 // rmsnorm.cu -- weightless RMSNorm rounded to bf16, the input of each MoE layer
-// of a stack: out = bf16(v / sqrt(mean(v^2) + eps)), fp32 arithmetic, IEEE
-// division and square root (no fast-math), round-to-nearest-even to bf16.
+// of a stack: out = bf16(v * r) with r = 1 / sqrt(mean(v^2) + eps), where r is
+// formed in fp32 with IEEE square root and IEEE division (no fast-math) and the
+// product is rounded to nearest-even bf16.
 #include "common.cuh"
 
 namespace moe {
