@@ -216,10 +216,98 @@ def step_inputs(cfg, workload, n, rank, dev):
     return syn.activations(n * T, cfg.H, 1 + 1000003 * rank, dev).view(n, T, cfg.H)
 
 
+DTYPE_DETAIL = {
+    1: "int4 codes decoded to f32, f32 FMA (CUDA cores); bf16 activations",
+    2: ("int4 codes against activations in 23-bit fixed point split into byte limbs (dp4a, "
+        "s32 accumulation, exact), limb sums combined in f64 and rounded once to f32"),
+    3: ("int4 codes converted to bf16 (gate/up) / f16 (down), tcgen05 MMA with f32 accumulation; "
+        "bf16 activations"),
+}
+
+
 def workload_name(cfg):
     return (f"{cfg.name}: T={cfg.T} per step, H={cfg.H} I={cfg.I} E={cfg.E}+1 shared "
             f"top-{cfg.k} n_group={cfg.n_group} topk_group={cfg.topk_group} rsf={cfg.rsf} "
             f"int{cfg.bits}, router bias {cfg.bias_kind}")
+
+
+
+def _staged_steps(L, bias, xs, cfg, T, flush, dev):
+    """Per-step device times of moe_layer_forward over the steps in xs [n, T, H]
+    (L2 flushed before each step, outside the events), replayed from one
+    captured graph; returns (step_ms [n], stage_ms [n, 5], idx [n, T, k])."""
+    stream = torch.cuda.current_stream()
+    n = xs.shape[0]
+    rc = L["rc"]
+    y = torch.empty((T, cfg.H), dtype=torch.float32, device=dev)
+    idx = torch.empty((n, T, cfg.k), dtype=torch.int32, device=dev)
+    ws = lib.Workspace(lib.moe_layer_workspace_bytes(T, cfg.H, cfg.I, rc), dev)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(lib.LAYER_EVENTS)] for _ in range(n)]
+    for e in (x for row in ev for x in row):
+        e.record(stream)
+
+    def step(i):
+        flush.fill_(i & 0xff)
+        lib.moe_layer_forward(xs[i], L["gate"], bias, rc, L["table"], L["shared"], cfg.bits, y=y,
+                              ws=ws, events=ev[i], idx_out=idx[i])
+
+    for i in range(min(n, 2)):  # warm-up outside the graph
+        step(i)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for i in range(n):
+            step(i)
+    g.replay()
+    torch.cuda.synchronize()
+    assert ws.flags() == 0
+    step_ms = np.array([ev[i][0].elapsed_time(ev[i][-1]) for i in range(n)])
+    stage_ms = np.array([[ev[i][s].elapsed_time(ev[i][s + 1]) for s in range(lib.LAYER_EVENTS - 1)]
+                         for i in range(n)])
+    del g
+    return step_ms, stage_ms, idx.cpu().numpy()
+
+
+def secondary_numbers(L, cfg, flush, dev, peaks, peak_kind, steps=8):
+    """Small batches with the Zipf-skewed router (T = 2, 8, 32) and the
+    4096-token prefill, on the same resident experts as the headline."""
+    H, I = cfg.H, cfg.I
+    ex_bytes = 2 * (I * H // 2 + I * 4) + (H * I // 2 + H * 4)
+    out = {"note": "same resident int4 experts as the headline; L2 flushed before every step; "
+                   "per-step CUDA events, medians over the steps"}
+    zipf = syn.router_bias(syn.SMALL_BATCH, 0, dev)
+    small = {}
+    for T in (2, 8, 32):
+        xs = syn.activations(steps * T, H, 7001 + T, dev).view(steps, T, H)
+        step_ms, _, idx = _staged_steps(L, zipf, xs, cfg, T, flush, dev)
+        uniq = np.array([len(np.unique(r[r >= 0])) for r in idx])
+        byts = (uniq + 1) * ex_bytes + cfg.E * H * 4
+        ms = float(np.median(step_ms))
+        gbs = float(np.median(byts / (step_ms * 1e-3))) / 1e9
+        small[f"T{T}"] = {"tokens_per_s": round(T / (ms * 1e-3), 1), "ms_per_step": round(ms, 5),
+                          "unique_experts": float(np.mean(uniq)),
+                          "expert_gbs": round(gbs, 1),
+                          "hbm_frac": round(gbs / peaks["hbm_gbs"], 4)}
+    out["small_batch_zipf"] = small
+    T = 4096
+    xs = syn.activations(3 * T, H, 7777, dev).view(3, T, H)
+    step_ms, stage_ms, idx = _staged_steps(L, L["bias"], xs, cfg, T, flush, dev)
+    pairs = np.array([int((r >= 0).sum()) for r in idx])
+    f1 = (pairs + T) * 2.0 * (2 * I) * H
+    f2 = (pairs + T) * 2.0 * I * H
+    t1 = float(np.median(f1 / (stage_ms[:, 2] * 1e-3))) / 1e12
+    t2 = float(np.median(f2 / (stage_ms[:, 3] * 1e-3))) / 1e12
+    ms = float(np.median(step_ms))
+    pk = peaks["bf16_tflops"]
+    out["prefill_T4096"] = {
+        "tokens_per_s": round(T / (ms * 1e-3), 1), "ms_per_step": round(ms, 4),
+        "layer_tflops": round(float(np.median((f1 + f2) / (step_ms * 1e-3))) / 1e12, 1),
+        "tc_ffn1_tflops": round(t1, 1), "tc_ffn1_frac": round(t1 / pk, 4),
+        "tc_ffn2_tflops": round(t2, 1), "tc_ffn2_frac": round(t2 / pk, 4),
+        "peak": pk, "peak_source": peak_kind + " (bf16 burst)",
+        "stage_ms_median": {n: round(float(np.median(stage_ms[:, s])), 4) for s, n in
+                            enumerate(["router", "bucket", "gate_up", "down", "combine"])}}
+    return out
 
 
 def run_ours(args, world, rank):
@@ -315,15 +403,27 @@ def run_ours(args, world, rank):
     gu_ms = stage_ms[:, 2]
     tokens = K * T * world
     value = job_tokens_per_s(T, K, world, total_ms)
-    if T < 64:
-        kern = ("gateup_decode" if T <= 8 else "gateup_gemv") + " (int4 gate+up GEMV + SwiGLU, CUDA cores)"
+    if T <= 2:
+        kern = "gateup_decode (int4 gate+up GEMV + SwiGLU, CUDA cores)"
         achieved = float(np.mean(gu_bytes / (gu_ms * 1e-3))) / 1e9
         roof = {"kernel": kern, "bound": "hbm", "achieved": round(achieved, 1),
                 "peak": peaks["hbm_gbs"], "peak_source": peak_kind, "unit": "GB/s",
                 "frac": round(achieved / peaks["hbm_gbs"], 4),
-                "traffic": measured_traffic("gateup_decode") if T <= 8 else None,
+                "traffic": measured_traffic("gateup_decode"),
                 "algorithmic_bytes_per_launch": int(np.mean(gu_bytes))}
-        launches = 3 if T <= 8 else 6
+        launches = 3
+    elif T <= 8:  # 3..8 tokens
+        # one persistent kernel per layer call: router, selection, experts, combine
+        kern = "decode_layer (router, int4 gate/up + SwiGLU, down + combine; CUDA cores, dp4a)"
+        layer_bytes = expert_bytes_step + cfg.E * H * 4
+        k_ms = stage_ms[:, 0]
+        achieved = float(np.mean(layer_bytes / (k_ms * 1e-3))) / 1e9
+        roof = {"kernel": kern, "bound": "hbm", "achieved": round(achieved, 1),
+                "peak": peaks["hbm_gbs"], "peak_source": peak_kind, "unit": "GB/s",
+                "frac": round(achieved / peaks["hbm_gbs"], 4),
+                "traffic": measured_traffic("decode_layer"),
+                "algorithmic_bytes_per_launch": int(np.mean(layer_bytes))}
+        launches = 1
     else:
         kern = "tc_ffn<1> (tcgen05 int4->bf16 grouped GEMM, gate+up + SwiGLU)"
         gu_flops = (pairs + T) * 2.0 * (2 * I) * H                  # 2 * M * N * K, gate and up
@@ -346,10 +446,8 @@ def run_ours(args, world, rank):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "f32" if T < 64 else "bf16",
-        "dtype_detail": ("int4 codes decoded to f32, f32 FMA (CUDA cores)" if T < 64 else
-                         "int4 codes converted to bf16 (gate/up) / f16 (down), tcgen05 MMA "
-                         "with f32 accumulation") + "; bf16 activations",
+        "dtype": "f32" if T <= 2 else ("s32" if T <= 8 else "bf16"),
+        "dtype_detail": DTYPE_DETAIL[1 if T <= 2 else (2 if T <= 8 else 3)],
         "data": "synthetic (seeded N(0,0.02) weights quantised on device; x ~ N(0,1) bf16)",
         "config": {"workload": workload_name(cfg), "tokens_per_step": T,
                    "l2": "flushed before every step (256 MB write, outside the timed events)",
@@ -368,8 +466,10 @@ def run_ours(args, world, rank):
         "load": {"quantize_s": round(L["load_s"], 3), "fp32_bytes": L["fp32_bytes"],
                  "int4_expert_bytes": L["expert_bytes"]},
     }
+    if args.workload == "decode" and not args.no_secondary and world == 1:
+        res["secondary"] = secondary_numbers(L, cfg, flush, dev, peaks, peak_kind)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        res["cpu_baseline"] = cpu_baseline(cfg, L, xs[W:W + 2], samples=1)
+        res["cpu_baseline"] = cpu_baseline(cfg, L, xs[W:W + 4], samples=4)
     return res
 
 
@@ -489,24 +589,33 @@ def _oracle_expert(orc, cfg, e, dev="cuda"):
     return orc.Expert(q[0][0], q[0][1], q[1][0], q[1][1], q[2][0], q[2][1], cfg.bits)
 
 
-def cpu_baseline(cfg, L, xs, samples=1):
-    """The oracle timed on the host cores on `samples` tokens of the workload."""
+def cpu_baseline(cfg, L, xs, samples=4):
+    """The oracle timed on the host cores on `samples` tokens of the workload,
+    once on one thread and once on every core (the oracle splits each expert
+    FFN's output rows over its threads; the results do not depend on the count)."""
     import oracle as orc
     gate = L["gate"].cpu().numpy()
     bias = L["bias"].cpu().numpy()
     xb = syn.bf16_bits(xs.reshape(-1, cfg.H)[:samples])
+    samples = xb.shape[0]
     r = orc.route(xb, gate, bias, cfg.k, cfg.n_group, cfg.topk_group, cfg.rsf)
     need = sorted(set(int(e) for e in r["idx"].reshape(-1)))
     experts = [_oracle_expert(orc, cfg, e) if e in need else None for e in range(cfg.E)]
     shared = _oracle_expert(orc, cfg, cfg.E)
-    t0 = time.perf_counter()
-    orc.layer(xb, gate, bias, experts, shared, cfg.H, cfg.I, cfg.k, cfg.n_group,
-              cfg.topk_group, cfg.rsf)
-    dt = time.perf_counter() - t0
-    return {"value": round(samples / dt, 4), "unit": "tokens/s", "cores": orc.num_threads(),
-            "kind": "oracle",
+    ncores = os.cpu_count() or 1
+    out = {}
+    for threads in (1, ncores):
+        orc.set_num_threads(threads)
+        t0 = time.perf_counter()
+        orc.layer(xb, gate, bias, experts, shared, cfg.H, cfg.I, cfg.k, cfg.n_group,
+                  cfg.topk_group, cfg.rsf)
+        out[threads] = samples / (time.perf_counter() - t0)
+    orc.set_num_threads(ncores)
+    return {"value": round(out[ncores], 4), "unit": "tokens/s", "cores": ncores,
+            "value_1_thread": round(out[1], 4), "kind": "oracle",
             "sample": f"{samples} token(s) of the GLM-scale decode layer through the fp64 C "
-                      f"oracle (routing + 9 experts), experts quantised beforehand (untimed)"}
+                      f"oracle (routing + 9 experts per token), on 1 thread and on {ncores}; "
+                      f"experts quantised beforehand (untimed)"}
 
 
 def run_reference(args, world, rank):
@@ -532,6 +641,8 @@ def run_reference(args, world, rank):
         return experts, r
 
     sh = expert(cfg.E)
+    ncores = os.cpu_count() or 1
+    orc.set_num_threads(ncores)
     times = []
     for i in range(K + W):
         experts, r = step(i)  # expert preparation (quantisation) is load time, untimed
@@ -549,13 +660,12 @@ def run_reference(args, world, rank):
         "steps": K, "warmup": W, "ms_per_step": round(total / K * 1e3, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
-        "config": {"workload": "GLM-scale MoE layer decode, T=1 per step, H=6144 I=2048 "
-                               "E=256+1 shared top-8 n_group=8 topk_group=4 rsf=2.5 int4",
-                   "tokens_per_step": 1},
-        "cpu_baseline": {"value": round(value, 4), "unit": "tokens/s", "cores": orc.num_threads(),
+        "config": {"workload": workload_name(cfg), "tokens_per_step": 1},
+        "cpu_baseline": {"value": round(value, 4), "unit": "tokens/s", "cores": ncores,
                          "kind": "oracle",
-                         "sample": "one token per step through the fp64 C oracle layer "
-                                   "(routing + 9 experts); expert quantisation untimed"},
+                         "sample": f"one token per step through the fp64 C oracle layer "
+                                   f"(routing + 9 experts, each expert's rows split over "
+                                   f"{ncores} threads); expert quantisation untimed"},
         "e2e": {"value": round(value, 4), "unit": "tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -569,6 +679,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="decode", choices=sorted(WORKLOADS) + sorted(STACKS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-secondary", action="store_true",
+                    help="skip the small-batch and prefill numbers of the decode workload")
     ap.add_argument("--repeat", type=int, default=10,
                     help="replays of the captured timed loop (the last one is reported)")
     args = ap.parse_args()

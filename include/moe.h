@@ -237,13 +237,15 @@ MOE_API moe_status moe_expert_ffn(const uint16_t *x, int64_t T, int64_t H, int64
  *   y       [T, H] fp32, overwritten
  *   idx_out [T, k] int32 and w_out [T, k] fp32, nullable (routing decision)
  * ws: moe_layer_workspace_bytes(T, H, I, cfg) bytes.
- * Paths: batches below 64 tokens run the CUDA-core GEMV kernels (T <= 8:
- * a fused router + bucketing launch and two streaming GEMV launches); from 64
- * tokens on, int4 layers run the tcgen05 tensor-core grouped GEMM (int4 codes
- * converted to bf16 / fp16 in registers and written to tensor memory, fp32
- * accumulation in tensor memory, h kept in fp16; H, I multiples of 128 only).
- * AUTO runs int8 and int2 layers on the CUDA-core path at every batch size
- * (up to 4096 tokens).  Both paths write one
+ * Paths (AUTO): one or two tokens run a fused router + bucketing launch and two
+ * streaming GEMV launches; 3..8 tokens run one persistent kernel (router,
+ * selection, gate/up, down and combine, every expert's rows split evenly over
+ * all SMs, exact integer dot products); from 9 tokens on, int4 layers run the
+ * tcgen05 tensor-core grouped GEMM (int4 codes converted to bf16 / fp16 in
+ * registers and written to tensor memory, fp32 accumulation in tensor memory,
+ * h kept in fp16; H, I multiples of 128 only).  MOE_PATH_GEMV forces the
+ * CUDA-core kernels.  AUTO runs int8 and int2 layers on the CUDA-core path at
+ * every batch size (up to 4096 tokens).  Both paths write one
  * fp32 partial per (token, expert) pair and add the partials of a token in a
  * fixed order, so y is bitwise reproducible run to run on either path (the two
  * paths round differently from each other).

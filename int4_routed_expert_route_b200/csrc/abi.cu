@@ -26,6 +26,12 @@ moe_status launch_route_fused(const uint16_t *, int64_t, int64_t, const float *,
                               int32_t *, int32_t *, int32_t *, int32_t *, int32_t *, int32_t *,
                               int32_t *, uint32_t *, int32_t *, int32_t, cudaStream_t);
 bool decode_ok(int64_t T, int64_t H, int64_t I, int32_t k, int32_t bits);
+bool fused_decode_ok(int64_t T, int64_t H, int64_t I, const moe_router_cfg *cfg, int32_t bits);
+moe_status run_fused_decode(const uint16_t *x, int64_t T, int64_t H, int64_t I, const float *gate,
+                            const float *bias, const moe_router_cfg *cfg, int32_t bits,
+                            const moe_expert *experts, const moe_expert *shared, float *y,
+                            int32_t accumulate, int32_t *idx_out, float *w_out, float *sb, float *h,
+                            float *yp, uint32_t *hdr, cudaStream_t stream);
 bool tc_ok(int64_t H, int64_t I);
 int32_t tc_tile_tokens();
 size_t tc_xs_bytes(int64_t T, int32_t k, int64_t H);
@@ -71,9 +77,11 @@ static bool cfg_ok(const moe_router_cfg *c) {
 }
 
 // Largest batch the CUDA-core path takes on; from kTensorMinT tokens on, AUTO
-// picks the tensor-core grouped GEMM.
+// picks the tensor-core grouped GEMM for int4 layers (measured: from about ten
+// tokens on a batch selects dozens of experts, and the grouped GEMM streams them
+// several times faster than the CUDA-core items kernels).
 static constexpr int64_t kGemvMaxT = 4096;
-static constexpr int64_t kTensorMinT = 64;
+static constexpr int64_t kTensorMinT = 9;
 
 bool plan_layer(int64_t T, int64_t H, int64_t I, const moe_router_cfg *cfg, int32_t path,
                 LayerPlan *p) {
@@ -289,6 +297,19 @@ moe_status moe_layer_forward_ex(const uint16_t *x, int64_t T, int64_t H, int64_t
     unsigned *counter = reinterpret_cast<unsigned *>(base + p.off_flags + 64);
     int32_t *tile_cnt = reinterpret_cast<int32_t *>(base + p.off_flags + 1024);
     float *logits = reinterpret_cast<float *>(base + p.off_part);
+
+    if (p.path == MOE_PATH_GEMV && T >= 3 && fused_decode_ok(T, H, I, cfg, weight_bits)) {
+        // 3..8 tokens: the whole layer in one persistent kernel whose blocks split
+        // every expert's rows evenly (the kernels below give each expert a fixed
+        // share of the blocks, which leaves most of them idle once a batch
+        // selects dozens of experts; measured crossover between 2 and 3 tokens)
+        rec(events, 0, stream);
+        st = run_fused_decode(x, T, H, I, gate, bias, cfg, weight_bits, experts, shared, y, accumulate,
+                              idx, w, logits, h, yp, flags, stream);
+        if (st != MOE_OK) return st;
+        for (int i = 1; i < 6; i++) rec(events, i, stream);
+        return MOE_OK;
+    }
 
     if (p.path == MOE_PATH_GEMV && route_fused_ok(T, H) && decode_ok(T, H, I, p.k, weight_bits)) {
         // decode-size batch: fused router + bucketing, then the two GEMV kernels

@@ -119,8 +119,8 @@ def test_host_side_path_and_size_contracts(so):
     # an empty batch is fine and launches nothing
     assert fwd(0, 6144, 2048, 4, m.PATH_AUTO) == 0
     # AUTO runs int8/int2 layers on the CUDA-core path: its workspace must fit in the one
-    # sized for AUTO (which plans the tensor path from 64 tokens on)
-    for T in (1, 8, 63, 64, 256, 4096):
+    # sized for AUTO (which plans the tensor path from 9 tokens on)
+    for T in (1, 2, 8, 9, 63, 64, 256, 4096):
         auto = m.moe_layer_workspace_bytes(T, 6144, 2048, cfg)
         gemv = m.moe_layer_workspace_bytes(T, 6144, 2048, cfg, m.PATH_GEMV)
         assert 0 < gemv <= auto, T
