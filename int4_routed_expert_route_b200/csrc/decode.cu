@@ -247,6 +247,9 @@ __device__ __forceinline__ unsigned ld_acquire(const unsigned *p) {
 }
 // Named barrier of the consumer warps (the producer warp never joins it).
 __device__ __forceinline__ void consumer_bar() { asm volatile("bar.sync 1, %0;" ::"n"(CTHREADS) : "memory"); }
+struct ConsumerBar {
+    static __device__ __forceinline__ void sync() { consumer_bar(); }
+};
 // Named barrier of consumers + producer (routed blocks, once routing is known).
 __device__ __forceinline__ void block_bar2() { asm volatile("bar.sync 2, %0;" ::"n"(THREADS) : "memory"); }
 // Barrier 3: the consumers signal (without waiting) that their router loads are
@@ -933,106 +936,20 @@ __device__ __forceinline__ void router_scores(const Args &a, Smem &S, int rb, in
 }
 
 // Group-limited top-k of every token from the published scores, by all
-// consumer threads at once: every (token, expert) finds its rank inside its
-// group (the two best make the group score), every (token, group) its rank
-// among the groups (the topk_group best are kept; ties to the lower group), and
-// every candidate of a kept group its rank among the candidates (descending
-// biased score, ties to the lower expert): rank r < k is slot r.  The same order
-// and tie rules as the warp-per-token router kernel.
+// consumer threads at once (select_tokens), after one bulk copy of the scores
+// into shared memory.
 __device__ __forceinline__ void select_block(const Args &a, Smem &S, uint32_t &ph, const Ctl &c) {
-    const int ctid = threadIdx.x;
-    const int T = a.T, E = a.E, k = a.k, ng = a.n_group, tkg = a.topk_group, gsz = E / ng;
-    const int TE = T * E;
+    const int TE = a.T * a.E;
     float *s_all = reinterpret_cast<float *>(S.red);  // [T][E]
     float *b_all = s_all + TE;                          // [T][E]
-    float *gtop = b_all + TE;                           // [T][ng][2]
-    float *gsc = gtop + T * ng * 2;                     // [T][ng]
-    int *kept = reinterpret_cast<int *>(gsc + T * ng);  // [T][topk_group] kept groups
-    int *pick = kept + T * tkg;                         // [T][k]
     {
         const void *src[1] = {a.sb};
         const uint32_t bytes[1] = {static_cast<uint32_t>((2 * TE * 4 + 15) & ~15)};  // the region is padded to 256 B
         uint8_t *dst[1] = {S.red};
         stage_copy(S, 1, src, bytes, dst, ph, c);
     }
-    for (int i = ctid; i < T * k; i += CTHREADS) pick[i] = -1;
-    consumer_bar();
-    if (ng > 1) {
-        for (int i = ctid; i < TE; i += CTHREADS) {
-            const int t = i / E, e = i - t * E, g = e / gsz;
-            const float *bt = b_all + t * E;
-            const float be = bt[e];
-            int rank = 0;
-#pragma unroll 8
-            for (int e2 = g * gsz; e2 < (g + 1) * gsz; e2++) {
-                const float o = bt[e2];
-                rank += (o > be) || (o == be && e2 < e);
-            }
-            if (rank < 2) gtop[(t * ng + g) * 2 + rank] = be;
-        }
-        consumer_bar();
-    }
-    for (int i = ctid; i < T * ng; i += CTHREADS) gsc[i] = ng == 1 ? 0.0f : gtop[2 * i] + gtop[2 * i + 1];
-    consumer_bar();
-    for (int i = ctid; i < T * ng; i += CTHREADS) {
-        const int t = i / ng, g = i - t * ng;
-        const float v = gsc[i];
-        int rank = 0;
-        for (int g2 = 0; g2 < ng; g2++) {
-            const float o = gsc[t * ng + g2];
-            rank += (o > v) || (o == v && g2 < g);
-        }
-        if (rank < tkg) kept[t * tkg + rank] = g;
-    }
-    consumer_bar();
-    // candidate ranks: four adjacent lanes per candidate split the comparisons
-    const int ncand = T * tkg * gsz;
-    for (int base = ctid & ~31; base < 4 * ncand; base += CTHREADS) {  // warp-uniform trip count
-        const int i0 = base + (ctid & 31);
-        const int i = i0 >> 2, part = i0 & 3;
-        const bool live = i < ncand;
-        int rank = 0, e = 0;
-        if (live) {
-            const int t = i / (tkg * gsz), rem = i - t * tkg * gsz;
-            e = kept[t * tkg + rem / gsz] * gsz + rem % gsz;
-            const float *bt = b_all + t * E;
-            const float be = bt[e];
-            for (int gi = part; gi < tkg; gi += 4) {  // part p compares with kept groups p, p + 4, ...
-                const int e0 = kept[t * tkg + gi] * gsz;
-#pragma unroll 8
-                for (int e2 = e0; e2 < e0 + gsz; e2++) {
-                    const float o = bt[e2];
-                    rank += (o > be) || (o == be && e2 < e);
-                }
-            }
-        }
-        rank += __shfl_xor_sync(0xffffffffu, rank, 1);
-        rank += __shfl_xor_sync(0xffffffffu, rank, 2);
-        if (live && part == 0 && rank < k) pick[(i / (tkg * gsz)) * k + rank] = e;
-    }
-    consumer_bar();
-    // weights: one warp per token, one lane per slot; the sum of the scores runs
-    // in slot order (the same fp32 rounding as one thread adding them)
-    const int warp = ctid >> 5, lane = ctid & 31;
-    for (int t = warp; t < T; t += NCW) {
-        const int *pk = pick + t * k;
-        const float *st = s_all + t * E;
-        const int pr = lane < k ? pk[lane] : -1;
-        const float sv = pr >= 0 ? st[pr] : 0.0f;
-        float sum = 0.0f;
-        for (int r = 0; r < k; r++) {
-            const float o = __shfl_sync(0xffffffffu, sv, r);
-            const int po = __shfl_sync(0xffffffffu, pr, r);
-            if (po >= 0) sum += o;
-        }
-        if (lane < k) {
-            S.sel_idx[t * k + lane] = pr;
-            S.sel_w[t * k + lane] = pr >= 0 ? (sv / sum) * a.rsf : 0.0f;
-        }
-        __syncwarp();
-        if (a.topp > 0.0f && a.topp < 1.0f && lane == 0)
-            finish_weights(st, pk, k, a.rsf, a.topp, S.sel_idx + t * k, S.sel_w + t * k);
-    }
+    select_tokens<ConsumerBar>(s_all, b_all, a.T, a.E, a.k, a.n_group, a.topk_group, a.rsf, a.topp, b_all + TE,
+                               S.sel_idx, S.sel_w, threadIdx.x, CTHREADS);
 }
 
 // Selection of every token, then the routed items; consumer threads only.
@@ -1339,8 +1256,9 @@ bool fused_decode_ok(int64_t T, int64_t H, int64_t I, const moe_router_cfg *cfg,
     // one row of gate + up must fit a ring stage
     if (2 * H * bits / 8 > dc::STAGE || I * bits / 8 > dc::STAGE) return false;
     // selection scratch inside the partials buffer: scores and biased scores,
-    // group tops and scores, kept groups, picks
-    const int64_t sel = static_cast<int64_t>(T) * (2 * cfg->n_experts + 3 * cfg->n_group + cfg->topk_group + cfg->top_k);
+    // then the selection's own scratch
+    const int64_t sel = static_cast<int64_t>(T) *
+                        (2 * cfg->n_experts + select_scratch_words(cfg->n_experts, cfg->top_k, cfg->n_group, cfg->topk_group));
     if (sel * 4 > dc::RED_BYTES) return false;
     return true;
 }

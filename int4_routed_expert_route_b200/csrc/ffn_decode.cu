@@ -230,6 +230,131 @@ __device__ __forceinline__ void chunk_fma(const uint32_t *wd, const f2 *act, f2 
     }
 }
 
+// int4 dot products on the integer pipe (dp4a).  A lane's 32 activations of
+// its chunk become integers X = round(x 2^F), one exponent F per lane and
+// chunk with max |X| in [2^21, 2^22), split into byte limbs X = X2 2^16 +
+// X1 2^8 + X0 (X0, X1 unsigned, X2 signed).  A weight word's nibbles split
+// into its even and odd codes (v & 0x0F0F0F0F, (v >> 4) & 0x0F0F0F0F), each
+// meeting the matching limb words in dp4a.  With the code bias folded in as
+// -8 sum(X), the lane's 32-code dot product sum (c - 8) X is exact in int32
+// (|.| < 32 * 8 * 2^22 = 2^30; the parts wrap modulo 2^32 on the way), and is
+// rounded once to fp32 and scaled by 2^-F (exact): 9 integer instructions per
+// 8 codes instead of 17 decode / f32x2 ones.  X is exact for bf16 inputs down
+// to 2^-14 of the chunk's largest magnitude, and within 2^-22 of it otherwise.
+struct Limbs4 {
+    uint32_t e[3][4], o[3][4];  // [limb][word]: limbs of columns 8w + 0,2,4,6 / 8w + 1,3,5,7
+    uint32_t bias;              // 8 * sum(X), modulo 2^32
+    float inv;                  // 2^-F
+};
+
+__device__ __forceinline__ uint32_t pack_limb(int32_t a, int32_t b, int32_t c, int32_t d, int l) {
+    const uint32_t sel = static_cast<uint32_t>(l | ((4 + l) << 4));
+    const uint32_t ab = __byte_perm(static_cast<uint32_t>(a), static_cast<uint32_t>(b), sel);
+    const uint32_t cd = __byte_perm(static_cast<uint32_t>(c), static_cast<uint32_t>(d), sel);
+    return __byte_perm(ab, cd, 0x5410);
+}
+
+template <typename Src>
+__device__ __forceinline__ void load_limbs4(const Src *src, bool have, Limbs4 &L) {
+    float v[32];
+#pragma unroll
+    for (int i = 0; i < 32; i++) v[i] = 0.0f;
+    if (have) {
+        if constexpr (sizeof(Src) == 2) {
+#pragma unroll
+            for (int i = 0; i < 4; i++) {
+                const uint4 q = *reinterpret_cast<const uint4 *>(src + 8 * i);
+                const uint32_t w4[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+                for (int j = 0; j < 4; j++) {
+                    v[8 * i + 2 * j] = __uint_as_float(w4[j] << 16);
+                    v[8 * i + 2 * j + 1] = __uint_as_float(w4[j] & 0xffff0000u);
+                }
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < 8; i++) {
+                const float4 q = *reinterpret_cast<const float4 *>(src + 4 * i);
+                v[4 * i] = q.x;
+                v[4 * i + 1] = q.y;
+                v[4 * i + 2] = q.z;
+                v[4 * i + 3] = q.w;
+            }
+        }
+    }
+    float m = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 32; i++) m = fmaxf(m, fabsf(v[i]));
+    int F = 0;
+    if (m > 0.0f) F = 21 - (static_cast<int>((__float_as_uint(m) >> 23) & 0xffu) - 127);
+    F = F > 126 ? 126 : (F < -126 ? -126 : F);
+    const float up = __uint_as_float(static_cast<uint32_t>(127 + F) << 23);
+    L.inv = __uint_as_float(static_cast<uint32_t>(127 - F) << 23);
+    int32_t X[32];
+    uint32_t sum = 0u;
+#pragma unroll
+    for (int i = 0; i < 32; i++) {
+        X[i] = __float2int_rn(v[i] * up);
+        sum += static_cast<uint32_t>(X[i]);
+    }
+    L.bias = 8u * sum;
+#pragma unroll
+    for (int w = 0; w < 4; w++)
+#pragma unroll
+        for (int l = 0; l < 3; l++) {
+            L.e[l][w] = pack_limb(X[8 * w], X[8 * w + 2], X[8 * w + 4], X[8 * w + 6], l);
+            L.o[l][w] = pack_limb(X[8 * w + 1], X[8 * w + 3], X[8 * w + 5], X[8 * w + 7], l);
+        }
+}
+
+// sum (c - 8) x over the lane's 32 codes (4 words), as fp32.
+__device__ __forceinline__ float dot4_dp4a(const uint32_t *wd, const Limbs4 &L) {
+    uint32_t a0 = 0u, a1 = 0u;
+    int32_t a2 = 0;
+#pragma unroll
+    for (int w = 0; w < 4; w++) {
+        const uint32_t ev = wd[w] & 0x0F0F0F0Fu, od = (wd[w] >> 4) & 0x0F0F0F0Fu;
+        asm("dp4a.u32.u32 %0, %1, %2, %0;" : "+r"(a0) : "r"(ev), "r"(L.e[0][w]));
+        asm("dp4a.u32.u32 %0, %1, %2, %0;" : "+r"(a0) : "r"(od), "r"(L.o[0][w]));
+        asm("dp4a.u32.u32 %0, %1, %2, %0;" : "+r"(a1) : "r"(ev), "r"(L.e[1][w]));
+        asm("dp4a.u32.u32 %0, %1, %2, %0;" : "+r"(a1) : "r"(od), "r"(L.o[1][w]));
+        asm("dp4a.u32.s32 %0, %1, %2, %0;" : "+r"(a2) : "r"(ev), "r"(L.e[2][w]));
+        asm("dp4a.u32.s32 %0, %1, %2, %0;" : "+r"(a2) : "r"(od), "r"(L.o[2][w]));
+    }
+    const uint32_t d = a0 + (a1 << 8) + (static_cast<uint32_t>(a2) << 16) - L.bias;
+    return __int2float_rn(static_cast<int32_t>(d)) * L.inv;
+}
+
+// A lane's activation registers for one token: dp4a limbs for int4, pre-scaled
+// fp32 pairs for the f32x2 decode of int8 / int2.
+template <int BITS>
+struct ActRegs {
+    f2 v[Chunk<BITS>::W * (Dec<BITS>::CPW / 2)];
+};
+template <>
+struct ActRegs<4> {
+    Limbs4 L;
+};
+
+template <int BITS, typename Src>
+__device__ __forceinline__ void load_act_regs(const Src *src, bool have, ActRegs<BITS> &r) {
+    if constexpr (BITS == 4) load_limbs4<Src>(src, have, r.L);
+    else load_act<BITS, Src>(src, have, r.v);
+}
+
+// decoded(chunk) . act of one lane chunk
+template <int BITS>
+__device__ __forceinline__ float chunk_dot(const uint32_t *wd, const ActRegs<BITS> &r) {
+    if constexpr (BITS == 4) {
+        return dot4_dp4a(wd, r.L);
+    } else {
+        f2 acc;
+        acc.v = 0ull;
+        chunk_fma<BITS>(wd, r.v, acc);
+        return f2_sum(acc);
+    }
+}
+
 // Per-lane asynchronous copy ring.  Every lane prefetches exactly the chunks it
 // will consume into its own shared-memory slots (cp.async), S-1 steps ahead, and
 // waits only for its own copy groups: no barrier is needed, and the prefetch
@@ -270,7 +395,6 @@ template <int BITS, int TG, int U>
 __global__ void __launch_bounds__(384, 1) gateup_decode(DecodeArgs a) {
     using D = Dec<BITS>;
     constexpr int CW = Chunk<BITS>::W;
-    constexpr int NP = CW * (D::CPW / 2);
     constexpr int V = U * 2 * TG;
     extern __shared__ __align__(16) uint8_t dsm_gu[];
     float *red = reinterpret_cast<float *>(dsm_gu);  // [DEC_RMAX][2][TG][KW]
@@ -288,7 +412,7 @@ __global__ void __launch_bounds__(384, 1) gateup_decode(DecodeArgs a) {
     int64_t r0, r1;
     dec_block_rows(dec_nseg(a), I, r0, r1);
 
-    f2 xs[TG][NP];
+    ActRegs<BITS> xs[TG];
     int64_t xs_seg = -1;
     for (int64_t r = r0; r < r1;) {
         const int64_t s = r / I;
@@ -307,7 +431,7 @@ __global__ void __launch_bounds__(384, 1) gateup_decode(DecodeArgs a) {
                     for (int t = 0; t < TG; t++) {
                         const bool have = active && t0 + t < g.n_tok;
                         const int64_t tok = have ? (g.toks ? g.toks[t0 + t] : t0 + t) : 0;
-                        load_act<BITS, uint16_t>(a.x + tok * H + col0, have, xs[t]);
+                        load_act_regs<BITS, uint16_t>(a.x + tok * H + col0, have, xs[t]);
                     }
                     xs_seg = s;
                 }
@@ -346,12 +470,8 @@ __global__ void __launch_bounds__(384, 1) gateup_decode(DecodeArgs a) {
 #pragma unroll
                         for (int mm = 0; mm < 2; mm++)
 #pragma unroll
-                            for (int t = 0; t < TG; t++) {
-                                f2 acc;
-                                acc.v = 0ull;
-                                if (active) chunk_fma<BITS>(wr[u][mm], xs[t], acc);
-                                v[(u * 2 + mm) * TG + t] = f2_sum(acc);
-                            }
+                            for (int t = 0; t < TG; t++)
+                                v[(u * 2 + mm) * TG + t] = active ? chunk_dot<BITS>(wr[u][mm], xs[t]) : 0.0f;
                     Bfly<V, 16>::run(v, lane);
                     if (bfly_writer<V>(lane)) {
                         const int idx = bfly_index<V>(lane);
@@ -398,7 +518,6 @@ template <int BITS, int TG, int U>
 __global__ void __launch_bounds__(TG == 1 ? 512 : 384, 1) down_decode(DecodeArgs a) {
     using D = Dec<BITS>;
     constexpr int CW = Chunk<BITS>::W;
-    constexpr int NP = CW * (D::CPW / 2);
     constexpr int V = U * TG;
     extern __shared__ __align__(16) uint8_t dsm_dn[];
     float *red = reinterpret_cast<float *>(dsm_dn);  // [DN_RMAX][TG][KW]
@@ -424,7 +543,7 @@ __global__ void __launch_bounds__(TG == 1 ? 512 : 384, 1) down_decode(DecodeArgs
         s_w[i] = a.w[i];
     }
 
-    f2 hs[TG][NP];
+    ActRegs<BITS> hs[TG];
     bool h_ready = false;  // h comes from the gate/up kernel: wait before the first read
     for (int64_t r = r0; r < r1;) {
         const int64_t s = r / H;
@@ -462,7 +581,7 @@ __global__ void __launch_bounds__(TG == 1 ? 512 : 384, 1) down_decode(DecodeArgs
 #pragma unroll
                 for (int t = 0; t < TG; t++) {
                     const bool have = active && t0 + t < g.n_tok;
-                    load_act<BITS, float>(a.h + (g.hrow + (have ? t0 + t : 0)) * I + col0, have, hs[t]);
+                    load_act_regs<BITS, float>(a.h + (g.hrow + (have ? t0 + t : 0)) * I + col0, have, hs[t]);
                 }
                 for (int st = 0; st < nsteps; st++) {
                     issue(st + DN_S - 1);
@@ -475,12 +594,7 @@ __global__ void __launch_bounds__(TG == 1 ? 512 : 384, 1) down_decode(DecodeArgs
 #pragma unroll
                     for (int u = 0; u < U; u++)
 #pragma unroll
-                        for (int t = 0; t < TG; t++) {
-                            f2 acc;
-                            acc.v = 0ull;
-                            if (active) chunk_fma<BITS>(wr[u], hs[t], acc);
-                            v[u * TG + t] = f2_sum(acc);
-                        }
+                        for (int t = 0; t < TG; t++) v[u * TG + t] = active ? chunk_dot<BITS>(wr[u], hs[t]) : 0.0f;
                     Bfly<V, 16>::run(v, lane);
                     if (bfly_writer<V>(lane)) {
                         const int idx = bfly_index<V>(lane);

@@ -207,8 +207,9 @@ __global__ void __launch_bounds__(SEL_WARPS * 32) route_select(SelArgs a) {
 // ---------------------------------------------------------------------------
 // Decode-size batches (T <= 8): logits, selection and batch-union bucketing in
 // one launch.  Every block computes one expert's logits; the last block to
-// finish (ticket counter in the workspace header) routes the tokens with its 8
-// warps and then buckets the (token, slot) pairs with a stable counting sort.
+// finish (ticket counter in the workspace header) routes the tokens with all
+// its threads (block-parallel ranks) and then buckets the (token, slot) pairs
+// with a stable counting sort.
 // The counter is reset by that block for the next call.
 // ---------------------------------------------------------------------------
 constexpr int FUSED_MAXT = 8;
@@ -231,15 +232,16 @@ struct FusedRouteArgs {
 // same outputs as the counting sort: list sorted by (expert, pair), tok, pos
 // (-1 for dropped slots), counts, offsets [E+1], ascending unique experts.
 // sm: 2 * P ints.
-__device__ void bucket_tiny(const int32_t *idx, int P, int k, int E, int32_t *counts, int32_t *offsets,
-                            int32_t *list, int32_t *tok, int32_t *pos, int32_t *unique,
+__device__ void bucket_tiny(const int32_t *idx_s, int32_t *idx_g, int P, int k, int E, int32_t *counts,
+                            int32_t *offsets, int32_t *list, int32_t *tok, int32_t *pos, int32_t *unique,
                             int32_t *n_unique, uint32_t *flags, int *sm) {
     int *pe = sm;         // [P] expert of each pair, -1 if dropped or invalid
     int *first = sm + P;  // [P] pair is the first of its expert
     const int tid = threadIdx.x;
     bool bad = false;
     for (int p = tid; p < P; p += blockDim.x) {
-        int e = __ldcg(idx + p);
+        int e = idx_s[p];
+        idx_g[p] = e;
         if (e >= E) {
             bad = true;
             e = -1;
@@ -310,22 +312,23 @@ __global__ void __launch_bounds__(RL_WARPS * 32) route_fused_small(FusedRouteArg
     if (threadIdx.x == 0) ticket = atomicAdd(a.counter, 1u);
     __syncthreads();
     if (ticket != gridDim.x - 1) return;
-    // 2. the last block: group-limited top-k of every token, then bucketing
+    // 2. the last block: group-limited top-k of every token (all its threads at
+    //    once), then bucketing
     __threadfence();
-    const int wid = threadIdx.x >> 5;
     float *s_all = dsm;               // [T][E]
     float *b_all = dsm + T * E;       // [T][E]
-    int *picks = reinterpret_cast<int *>(b_all + T * E);  // [8][32]
     for (int64_t i = threadIdx.x; i < T * E; i += blockDim.x) {
         s_all[i] = __ldcg(s_g + i);
         b_all[i] = __ldcg(b_g + i);
     }
     __syncthreads();
-    for (int64_t t = wid; t < T; t += RL_WARPS)
-        select_core(a.sel, t, s_all + t * E, b_all + t * E, picks + wid * 32);
-    __syncthreads();
-    bucket_tiny(a.sel.idx_out, static_cast<int>(a.sel.T * a.sel.k), a.sel.k, E, a.counts, a.offsets,
-                a.list, a.tok, a.pos, a.unique, a.n_unique, a.flags, reinterpret_cast<int *>(dsm));
+    const int ng = a.sel.n_group, tkg = a.sel.topk_group, k = a.sel.k;
+    float *scratch = b_all + T * E;
+    int32_t *idx_s = reinterpret_cast<int32_t *>(scratch + T * select_scratch_words(E, k, ng, tkg));  // [T][k]
+    select_tokens<BlockBar>(s_all, b_all, static_cast<int>(T), E, k, ng, tkg, a.sel.rsf, a.sel.topp, scratch,
+                            idx_s, a.sel.w_out, threadIdx.x, blockDim.x);
+    bucket_tiny(idx_s, a.sel.idx_out, static_cast<int>(T * k), k, E, a.counts, a.offsets, a.list, a.tok,
+                a.pos, a.unique, a.n_unique, a.flags, reinterpret_cast<int *>(dsm));
     for (int i = threadIdx.x; i < a.n_zero; i += blockDim.x) a.zero_cnt[i] = 0;
     if (threadIdx.x == 0) *a.counter = 0u;
 }
@@ -408,7 +411,10 @@ moe_status launch_route_fused(const uint16_t *x, int64_t T, int64_t H, const flo
     a.zero_cnt = zero_cnt;
     a.n_zero = n_zero;
     const int E = cfg->n_experts;
-    size_t smem = static_cast<size_t>(2 * T * E + RL_WARPS * 32) * sizeof(float);
+    // scores, biased scores, the selection's scratch and the selected indices
+    size_t smem = static_cast<size_t>(
+                      2 * T * E + T * (select_scratch_words(E, cfg->top_k, cfg->n_group, cfg->topk_group) + cfg->top_k)) *
+                  sizeof(float);
     const size_t bsm = static_cast<size_t>(2 * T * cfg->top_k) * sizeof(int);  // bucket_tiny
     if (bsm > smem) smem = bsm;
     if (smem > 48 * 1024 &&

@@ -190,4 +190,250 @@ static __device__ void select_core(const SelArgs &a, int64_t t, const float *s_s
     else select_core_j<32>(a, t, s_sm, b_sm, pick);
 }
 
+// Block-parallel group-limited top-k of T tokens from their scores s_all and
+// biased scores b_all ([T][E] in shared memory), by nthr threads at once (a
+// multiple of 32; Bar::sync() joins them): every (token, expert) finds its rank
+// inside its group (the two best make the group score), every (token, group)
+// its rank among the groups (the topk_group best are kept, ties to the lower
+// group), and every candidate of a kept group its rank among the candidates
+// (descending biased score, ties to the lower expert; four adjacent lanes split
+// the comparisons): rank r < k is slot r.  Then the weights (finish_weights'
+// arithmetic, one warp per token with the sum in slot order).  The same order
+// and tie rules as select_core.  scratch holds T * (3 n_group + topk_group + k)
+// words; idx_out / w_out [T][k] may be shared or global memory.
+template <class Bar>
+static __device__ __forceinline__ void select_block_ranks(const float *s_all, const float *b_all, int T, int E,
+                                                          int k, int ng, int tkg, float rsf, float topp,
+                                                          float *scratch, int32_t *idx_out, float *w_out, int tid,
+                                                          int nthr) {
+    const int gsz = E / ng, TE = T * E;
+    float *gtop = scratch;                              // [T][ng][2]
+    float *gsc = gtop + T * ng * 2;                     // [T][ng]
+    int *kept = reinterpret_cast<int *>(gsc + T * ng);  // [T][tkg] kept groups
+    int *pick = kept + T * tkg;                         // [T][k]
+    for (int i = tid; i < T * k; i += nthr) pick[i] = -1;
+    if (ng > 1) {
+        for (int i = tid; i < TE; i += nthr) {
+            const int t = i / E, e = i - t * E, g = e / gsz;
+            const float *bt = b_all + t * E;
+            const float be = bt[e];
+            int rank = 0;
+#pragma unroll 8
+            for (int e2 = g * gsz; e2 < (g + 1) * gsz; e2++) {
+                const float o = bt[e2];
+                rank += (o > be) || (o == be && e2 < e);
+            }
+            if (rank < 2) gtop[(t * ng + g) * 2 + rank] = be;
+        }
+    }
+    Bar::sync();
+    for (int i = tid; i < T * ng; i += nthr) gsc[i] = ng == 1 ? 0.0f : gtop[2 * i] + gtop[2 * i + 1];
+    Bar::sync();
+    for (int i = tid; i < T * ng; i += nthr) {
+        const int t = i / ng, g = i - t * ng;
+        const float v = gsc[i];
+        int rank = 0;
+        for (int g2 = 0; g2 < ng; g2++) {
+            const float o = gsc[t * ng + g2];
+            rank += (o > v) || (o == v && g2 < g);
+        }
+        if (rank < tkg) kept[t * tkg + rank] = g;
+    }
+    Bar::sync();
+    const int ncand = T * tkg * gsz;
+    for (int base = tid & ~31; base < 4 * ncand; base += nthr) {  // warp-uniform trip count
+        const int i0 = base + (tid & 31);
+        const int i = i0 >> 2, part = i0 & 3;
+        const bool live = i < ncand;
+        int rank = 0, e = 0;
+        if (live) {
+            const int t = i / (tkg * gsz), rem = i - t * tkg * gsz;
+            e = kept[t * tkg + rem / gsz] * gsz + rem % gsz;
+            const float *bt = b_all + t * E;
+            const float be = bt[e];
+            for (int gi = part; gi < tkg; gi += 4) {  // part p compares with kept groups p, p + 4, ...
+                const int e0 = kept[t * tkg + gi] * gsz;
+#pragma unroll 8
+                for (int e2 = e0; e2 < e0 + gsz; e2++) {
+                    const float o = bt[e2];
+                    rank += (o > be) || (o == be && e2 < e);
+                }
+            }
+        }
+        rank += __shfl_xor_sync(0xffffffffu, rank, 1);
+        rank += __shfl_xor_sync(0xffffffffu, rank, 2);
+        if (live && part == 0 && rank < k) pick[(i / (tkg * gsz)) * k + rank] = e;
+    }
+    Bar::sync();
+    const int warp = tid >> 5, lane = tid & 31;
+    for (int t = warp; t < T; t += nthr >> 5) {
+        const int *pk = pick + t * k;
+        const float *st = s_all + t * E;
+        const int pr = lane < k ? pk[lane] : -1;
+        const float sv = pr >= 0 ? st[pr] : 0.0f;
+        float sum = 0.0f;
+        for (int r = 0; r < k; r++) {
+            const float o = __shfl_sync(0xffffffffu, sv, r);
+            const int po = __shfl_sync(0xffffffffu, pr, r);
+            if (po >= 0) sum += o;
+        }
+        if (lane < k) {
+            idx_out[t * k + lane] = pr;
+            w_out[t * k + lane] = pr >= 0 ? (sv / sum) * rsf : 0.0f;
+        }
+        __syncwarp();
+        if (topp > 0.0f && topp < 1.0f && lane == 0) finish_weights(st, pk, k, rsf, topp, idx_out + t * k, w_out + t * k);
+    }
+    Bar::sync();
+}
+
+struct BlockBar {
+    static __device__ __forceinline__ void sync() { __syncthreads(); }
+};
+
+// Order-preserving 32-bit key of an fp32 value (a larger value has a larger
+// unsigned key; -0 is folded into +0 so that the keys tie where the fp32
+// comparison does), and its inverse.
+static __device__ __forceinline__ uint32_t order_key(float v) {
+    const uint32_t u = __float_as_uint(v + 0.0f);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+static __device__ __forceinline__ float key_value(uint32_t key) {
+    return __uint_as_float((key & 0x80000000u) ? (key & 0x7fffffffu) : ~key);
+}
+
+constexpr int SELW_MAXC = 8;  // candidates per lane of select_block_warps
+
+// select_block_warps applies when every group fits one warp's lanes, the group
+// scores fit one warp and a token's candidates fit SELW_MAXC per lane.
+static __host__ __device__ __forceinline__ bool select_warps_fit(int E, int k, int ng, int tkg) {
+    const int gsz = E / ng, qpg = (gsz + 31) / 32;
+    if (k > 32) return false;
+    if (ng == 1) return qpg <= SELW_MAXC;
+    return gsz <= 32 && ng <= 32 && tkg * qpg <= SELW_MAXC;
+}
+
+// Group-limited top-k of T tokens with warp reductions, the same result as
+// select_block_ranks in two barrier phases:
+//  1. one warp per (token, group): the group's two largest biased scores by two
+//     unsigned max-reductions over order keys (the second is the first again
+//     when two lanes hold it); lane 0 stores their fp32 sum;
+//  2. one warp per token: lane g ranks group g among the group scores (ties to
+//     the lower group) and a ballot gives the kept groups; every lane then holds
+//     the candidates j = lane, lane + 32, ... of each kept group (ascending
+//     expert order), and k rounds take the largest key (max-reduction) and,
+//     among the lanes holding it, the lowest expert (min-reduction): round r
+//     gives slot r.  Then the weights as in select_block_ranks.
+// Its rounds are serial, so it pays off where several tokens run side by side.
+// scratch: T * (n_group + k) words.
+template <class Bar>
+static __device__ __forceinline__ void select_block_warps(const float *s_all, const float *b_all, int T, int E,
+                                                          int k, int ng, int tkg, float rsf, float topp,
+                                                          float *scratch, int32_t *idx_out, float *w_out, int tid,
+                                                          int nthr) {
+    const int gsz = E / ng;
+    const int warp = tid >> 5, lane = tid & 31, nwarps = nthr >> 5;
+    constexpr int NONE = 0x7fffffff;
+    float *gsc = scratch;                               // [T][ng]
+    int *pick = reinterpret_cast<int *>(gsc + T * ng);  // [T][k]
+    if (ng > 1) {
+        for (int task = warp; task < T * ng; task += nwarps) {
+            const int t = task / ng, g = task - t * ng;
+            const uint32_t key = lane < gsz ? order_key(b_all[t * E + g * gsz + lane]) : 0u;
+            const uint32_t m1 = __reduce_max_sync(0xffffffffu, key);
+            const uint32_t hold = __ballot_sync(0xffffffffu, key == m1);
+            const uint32_t m2 = __popc(hold) >= 2 ? m1 : __reduce_max_sync(0xffffffffu, key == m1 ? 0u : key);
+            if (lane == 0) gsc[task] = key_value(m1) + key_value(m2);
+        }
+        Bar::sync();
+    }
+    for (int t = warp; t < T; t += nwarps) {
+        const float *bt = b_all + t * E;
+        uint32_t kept = 1u;
+        if (ng > 1) {
+            const float v = lane < ng ? gsc[t * ng + lane] : 0.0f;
+            int rank = 0;
+            for (int g2 = 0; g2 < ng; g2++) {
+                const float o = __shfl_sync(0xffffffffu, v, g2);
+                rank += (o > v) || (o == v && g2 < lane);
+            }
+            kept = __ballot_sync(0xffffffffu, lane < ng && rank < tkg);
+        }
+        // slot c of a lane: kept group number c / qpg (ascending), j = lane + 32 (c % qpg)
+        const int qpg = (gsz + 31) >> 5;
+        uint32_t ck[SELW_MAXC], avail = 0u, km = kept;
+        int ce[SELW_MAXC], g = -1, q = qpg;
+#pragma unroll
+        for (int c = 0; c < SELW_MAXC; c++) {
+            if (q == qpg) {
+                q = 0;
+                g = km ? __ffs(km) - 1 : -1;
+                km &= km - 1;
+            }
+            const int j = lane + 32 * q;
+            const bool ok = g >= 0 && j < gsz;
+            ck[c] = ok ? order_key(bt[g * gsz + j]) : 0u;
+            ce[c] = ok ? g * gsz + j : NONE;
+            avail |= static_cast<uint32_t>(ok) << c;
+            q++;
+        }
+        int mine = -1;
+        for (int r = 0; r < k; r++) {
+            uint32_t bk = 0u;
+            int be = NONE;
+#pragma unroll
+            for (int c = 0; c < SELW_MAXC; c++)
+                if (((avail >> c) & 1u) && (ck[c] > bk || (ck[c] == bk && ce[c] < be))) {
+                    bk = ck[c];
+                    be = ce[c];
+                }
+            const uint32_t top = __reduce_max_sync(0xffffffffu, bk);
+            const int win = static_cast<int>(
+                __reduce_min_sync(0xffffffffu, bk == top ? static_cast<uint32_t>(be) : static_cast<uint32_t>(NONE)));
+#pragma unroll
+            for (int c = 0; c < SELW_MAXC; c++)
+                if (ce[c] == win) avail &= ~(1u << c);
+            if (lane == r) mine = win == NONE ? -1 : win;
+        }
+        if (lane < k) pick[t * k + lane] = mine;
+        const float *st = s_all + t * E;
+        const float sv = mine >= 0 ? st[mine] : 0.0f;
+        float sum = 0.0f;
+        for (int r = 0; r < k; r++) {
+            const float o = __shfl_sync(0xffffffffu, sv, r);
+            if (__shfl_sync(0xffffffffu, mine, r) >= 0) sum += o;
+        }
+        if (lane < k) {
+            idx_out[t * k + lane] = mine;
+            w_out[t * k + lane] = mine >= 0 ? (sv / sum) * rsf : 0.0f;
+        }
+        __syncwarp();
+        if (topp > 0.0f && topp < 1.0f && lane == 0)
+            finish_weights(st, pick + t * k, k, rsf, topp, idx_out + t * k, w_out + t * k);
+    }
+    Bar::sync();
+}
+
+// Words of selection scratch per token (either form of select_tokens).
+static __host__ __device__ __forceinline__ int select_scratch_words(int E, int k, int ng, int tkg) {
+    (void)E;
+    return 3 * ng + tkg + k;
+}
+
+// Group-limited top-k of T tokens by nthr threads (Bar::sync() joins them):
+// from three tokens on the warp-reduction form where the configuration fits it
+// and has at most 16 groups (about three times faster than the rank form at
+// eight tokens of 256 experts in 8 groups), else the rank form (the faster of
+// the two for one or two tokens, and with many small groups).
+// scratch: T * select_scratch_words() words.
+template <class Bar>
+static __device__ __forceinline__ void select_tokens(const float *s_all, const float *b_all, int T, int E, int k,
+                                                     int ng, int tkg, float rsf, float topp, float *scratch,
+                                                     int32_t *idx_out, float *w_out, int tid, int nthr) {
+    if (T >= 3 && ng <= 16 && select_warps_fit(E, k, ng, tkg))
+        select_block_warps<Bar>(s_all, b_all, T, E, k, ng, tkg, rsf, topp, scratch, idx_out, w_out, tid, nthr);
+    else
+        select_block_ranks<Bar>(s_all, b_all, T, E, k, ng, tkg, rsf, topp, scratch, idx_out, w_out, tid, nthr);
+}
+
 }  // namespace moe

@@ -45,9 +45,15 @@ def stack_check(lib, orc, cfg, n_layers, T, seed):
     for l, OL in enumerate(oracle):
         xb, _ = orc.rmsnorm_bf16(r, 1e-6)
         # the layer input: bf16 of the same norm, rounded from fp32 on the GPU
-        # and from fp64 in the oracle -> equal up to one bf16 ulp
+        # and from fp64 in the oracle -> equal up to one bf16 ulp on layer 0.
+        # After that the two chains carry different residuals: one ulp flipped
+        # by that rounding (0.4% of one input element) moves the layer's output
+        # by up to ~1e-4 of max |y| (a single-layer run on identical inputs
+        # agrees to 1e-6), so later inputs also get the layer tolerance, scaled
+        # by the norm like everything else
         gv, ov = _bf16_bits_to_f64(gpu_li[l]), _bf16_bits_to_f64(xb)
-        assert np.all(np.abs(gv - ov) <= np.abs(ov) * 2.0 ** -7 + 1e-30), l
+        allow = np.abs(ov) * 2.0 ** -7 + (TOL * l * np.max(np.abs(ov)) if l else 1e-30)
+        assert np.all(np.abs(gv - ov) <= allow), (l, float(np.max(np.abs(gv - ov) - allow)))
         ro = OL.route(xb)
         fl = flagged(ro)
         use_idx, use_w = ro["idx"].copy(), ro["w"].copy()
@@ -69,8 +75,11 @@ def test_stack_tiny_three_layers(lib, orc):
     stack_check(lib, orc, syn.TINY, n_layers=3, T=4, seed=11)
 
 
-def test_stack_glm_two_layers_decode(lib, orc):
-    stack_check(lib, orc, syn.DECODE, n_layers=2, T=1, seed=12)
+@pytest.mark.parametrize("T", [1, 4])
+def test_stack_glm_two_layers_decode(lib, orc, T):
+    """T = 1 runs the fused router + streaming GEMV kernels, T = 4 the fused
+    decode-layer kernel, both two GLM-scale layers deep."""
+    stack_check(lib, orc, syn.DECODE, n_layers=2, T=T, seed=12)
 
 
 # ---------------------------------------------------------------------------
