@@ -41,7 +41,7 @@ moe_status run_tc_layer(const uint16_t *x, int64_t T, int64_t H, int64_t I, int3
                         const float *w, void *h, void *xs, float *yp, unsigned *counters,
                         uint32_t *flags, cudaStream_t stream, cudaEvent_t ev_down);
 moe_status run_decode_layer(const uint16_t *x, int64_t T, int64_t H, int64_t I, int32_t k,
-                            int32_t bits, const moe_expert *experts, const moe_expert *shared,
+                            int32_t bits, const moe_expert *experts, int32_t n_experts, const moe_expert *shared,
                             const int32_t *unique, const int32_t *n_unique, const int32_t *offsets,
                             const int32_t *tok, const int32_t *pos, const int32_t *idx,
                             const float *w, float *h, float *yp, int32_t *tile_cnt, float *y,
@@ -320,7 +320,7 @@ moe_status moe_layer_forward_ex(const uint16_t *x, int64_t T, int64_t H, int64_t
         if (st != MOE_OK) return st;
         rec(events, 1, stream);
         rec(events, 2, stream);
-        st = run_decode_layer(x, T, H, I, p.k, weight_bits, experts, shared, unique, nunique,
+        st = run_decode_layer(x, T, H, I, p.k, weight_bits, experts, cfg->n_experts, shared, unique, nunique,
                               offsets, tok, pos, idx, w, h, yp, tile_cnt, y, accumulate, flags,
                               stream, events ? events[3] : nullptr);
         if (st != MOE_OK) return st;

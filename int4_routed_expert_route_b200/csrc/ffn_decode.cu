@@ -45,6 +45,7 @@ struct DecodeArgs {
     float *yp;        // [T*k + T, H] fp32 per-pair down outputs
     int32_t *tile_cnt;  // [H / 64] completion counters (zero between calls)
     int32_t accumulate;
+    int32_t n_experts;
     int32_t kw, rg;   // K-slice warps, row groups (blockDim = 32 * kw * rg)
     int32_t rows_pb;  // down: max output rows per block (smem sizing)
     uint32_t *flags;
@@ -57,11 +58,16 @@ struct DSeg {
     int64_t hrow;
 };
 
+// Segments: the shared expert first when present, then the routed experts.
+// With one token the routed segments are the k selection slots themselves
+// (slot p is h / yp row p; a slot dropped by the expert top-p, or holding an
+// index out of range, is an empty segment), read straight from the selection:
+// no bucketing.  Otherwise they are the batch's unique experts in ascending
+// order, with their token lists from the bucketing.
 __device__ __forceinline__ int64_t dec_nseg(const DecodeArgs &a) {
-    return static_cast<int64_t>(*a.n_unique) + (a.shared ? 1 : 0);
+    return (a.T == 1 ? static_cast<int64_t>(a.k) : static_cast<int64_t>(*a.n_unique)) + (a.shared ? 1 : 0);
 }
 
-// Segment 0 is the shared expert when present, then the unique routed experts.
 __device__ __forceinline__ DSeg dec_seg(const DecodeArgs &a, int64_t s) {
     DSeg g;
     if (a.shared) {
@@ -73,6 +79,16 @@ __device__ __forceinline__ DSeg dec_seg(const DecodeArgs &a, int64_t s) {
             return g;
         }
         s -= 1;
+    }
+    if (a.T == 1) {
+        const int e = a.idx[s];
+        const bool valid = e >= 0 && e < a.n_experts;
+        if (e >= a.n_experts) raise_flag(a.flags, MOE_FLAG_BAD_EXPERT_INDEX);
+        g.ex = valid ? a.experts + e : nullptr;
+        g.toks = nullptr;
+        g.n_tok = valid ? 1 : 0;
+        g.hrow = s;
+        return g;
     }
     const int e = a.unique[s];
     const int o0 = a.offsets[e], o1 = a.offsets[e + 1];
@@ -407,18 +423,33 @@ __global__ void __launch_bounds__(384, 1) gateup_decode(DecodeArgs a) {
     const int64_t chunk = static_cast<int64_t>(kw) * 32 + lane;
     const bool active = chunk * D::CH < rb;
     const int64_t col0 = chunk * D::NC;
-    griddep_wait();    // routing of this batch (previous kernel)
-    griddep_launch();  // the down kernel may start its weight prologue
-    int64_t r0, r1;
-    dec_block_rows(dec_nseg(a), I, r0, r1);
-
+    // One token: its activations and the block's rows are known before the
+    // routing is (every expert sees token 0; the segments are the shared
+    // expert and the k routed slots), so the activations load while the router
+    // still runs, and the shared expert's blocks do all their work then.
     ActRegs<BITS> xs[TG];
     int64_t xs_seg = -1;
+    const bool one_token = a.T == 1;
+    int64_t r0, r1;
+    if (one_token) {
+        dec_block_rows(dec_nseg(a), I, r0, r1);
+        load_act_regs<BITS, uint16_t>(a.x + col0, active, xs[0]);
+        if (!(a.shared && r0 < r1 && r1 <= I)) griddep_wait();  // routing of this batch
+    } else {
+        griddep_wait();
+        dec_block_rows(dec_nseg(a), I, r0, r1);
+    }
+    griddep_launch();  // the down kernel may start its weight prologue
+
     for (int64_t r = r0; r < r1;) {
         const int64_t s = r / I;
         const int64_t run_end = min(r1, (s + 1) * I);
         const int64_t i_begin = r - s * I;
         const DSeg g = dec_seg(a, s);
+        if (!g.ex) {  // an empty slot
+            r = run_end;
+            continue;
+        }
         const moe_qmat mg = g.ex->gate, mu = g.ex->up;
         const bool ok = dqmat_ok(mg, BITS, I, H) && dqmat_ok(mu, BITS, I, H);
         if (!ok && threadIdx.x == 0) raise_flag(a.flags, MOE_FLAG_BAD_EXPERT_SHAPE);
@@ -426,15 +457,6 @@ __global__ void __launch_bounds__(384, 1) gateup_decode(DecodeArgs a) {
             const int m = static_cast<int>(run_end - r - sub < DEC_RMAX ? run_end - r - sub : DEC_RMAX);
             const int64_t ib = i_begin + sub;  // first row (within the expert) of this sub-run
             for (int64_t t0 = 0; t0 < g.n_tok; t0 += TG) {
-                if (xs_seg != s || g.n_tok > TG) {
-#pragma unroll
-                    for (int t = 0; t < TG; t++) {
-                        const bool have = active && t0 + t < g.n_tok;
-                        const int64_t tok = have ? (g.toks ? g.toks[t0 + t] : t0 + t) : 0;
-                        load_act_regs<BITS, uint16_t>(a.x + tok * H + col0, have, xs[t]);
-                    }
-                    xs_seg = s;
-                }
                 const int nmy = rg < m ? (m - rg + RG - 1) / RG : 0;
                 const int nsteps = (nmy + U - 1) / U;
                 uint8_t *ring = ring_base + static_cast<size_t>(warp) * (GU_S * U * 2 * 32 * D::CH);
@@ -454,7 +476,23 @@ __global__ void __launch_bounds__(384, 1) gateup_decode(DecodeArgs a) {
                     cp_async_commit();
                 };
 #pragma unroll
-                for (int st = 0; st < GU_S - 1; st++) issue(st);
+                for (int st = 0; st < GU_S - 1; st++) issue(st);  // weights first, then the activations
+                if (!one_token && (xs_seg != s || g.n_tok > TG)) {
+#pragma unroll
+                    for (int t = 0; t < TG; t++) {
+                        const bool have = active && t0 + t < g.n_tok;
+                        const int64_t tok = have ? (g.toks ? g.toks[t0 + t] : t0 + t) : 0;
+                        load_act_regs<BITS, uint16_t>(a.x + tok * H + col0, have, xs[t]);
+                    }
+                    xs_seg = s;
+                }
+                // the epilogue's row scales, loaded while the rows stream
+                float pre_g = 0.0f, pre_u = 0.0f;
+                if (static_cast<int>(threadIdx.x) < m * TG) {
+                    const int64_t row = ib + threadIdx.x / TG;
+                    pre_g = mg.scale[row];
+                    pre_u = mu.scale[row];
+                }
                 for (int st = 0; st < nsteps; st++) {
                     issue(st + GU_S - 1);
                     cp_async_wait<GU_S - 1>();
@@ -491,7 +529,8 @@ __global__ void __launch_bounds__(384, 1) gateup_decode(DecodeArgs a) {
                             su += red[((lr * 2 + 1) * TG + t) * KW + w];
                         }
                         const int64_t row = ib + lr;
-                        const float gv = sg * mg.scale[row], uv = su * mu.scale[row];
+                        const bool pre = q == static_cast<int>(threadIdx.x);
+                        const float gv = sg * (pre ? pre_g : mg.scale[row]), uv = su * (pre ? pre_u : mu.scale[row]);
                         a.h[(g.hrow + t0 + t) * I + row] = silu(gv) * uv;
                     }
                 }
@@ -539,7 +578,8 @@ __global__ void __launch_bounds__(TG == 1 ? 512 : 384, 1) down_decode(DecodeArgs
     __shared__ int32_t s_pos[8 * 32];
     __shared__ float s_w[8 * 32];
     for (int i = threadIdx.x; i < T * a.k; i += blockDim.x) {
-        s_pos[i] = a.pos[i];
+        // one token: slot p is row p unless dropped (see dec_seg)
+        s_pos[i] = T == 1 ? (a.idx[i] >= 0 && a.idx[i] < a.n_experts ? i : -1) : a.pos[i];
         s_w[i] = a.w[i];
     }
 
@@ -550,8 +590,8 @@ __global__ void __launch_bounds__(TG == 1 ? 512 : 384, 1) down_decode(DecodeArgs
         const int64_t run_end = min(r1, (s + 1) * H);
         const int64_t j_begin = r - s * H;
         const DSeg g = dec_seg(a, s);
-        const moe_qmat md = g.ex->down;
-        const bool ok = dqmat_ok(md, BITS, H, I);
+        const moe_qmat md = g.ex ? g.ex->down : moe_qmat{};
+        const bool ok = !g.ex || dqmat_ok(md, BITS, H, I);  // an empty slot computes nothing but counts its rows
         if (!ok && threadIdx.x == 0) raise_flag(a.flags, MOE_FLAG_BAD_EXPERT_SHAPE);
         for (int64_t sub = 0; sub < run_end - r; sub += DN_RMAX) {
             const int m = static_cast<int>(run_end - r - sub < DN_RMAX ? run_end - r - sub : DN_RMAX);
@@ -578,6 +618,8 @@ __global__ void __launch_bounds__(TG == 1 ? 512 : 384, 1) down_decode(DecodeArgs
                     griddep_wait();
                     h_ready = true;
                 }
+                float pre_s = 0.0f;  // the epilogue's row scale, loaded while the rows stream
+                if (static_cast<int>(threadIdx.x) < m * TG) pre_s = md.scale[jb + threadIdx.x / TG];
 #pragma unroll
                 for (int t = 0; t < TG; t++) {
                     const bool have = active && t0 + t < g.n_tok;
@@ -611,7 +653,7 @@ __global__ void __launch_bounds__(TG == 1 ? 512 : 384, 1) down_decode(DecodeArgs
                         float d = 0.f;
                         for (int w = 0; w < KW; w++) d += red[(lr * TG + t) * KW + w];
                         const int64_t j = jb + lr;
-                        a.yp[(g.hrow + t0 + t) * H + j] = d * md.scale[j];
+                        a.yp[(g.hrow + t0 + t) * H + j] = d * (q == static_cast<int>(threadIdx.x) ? pre_s : md.scale[j]);
                     }
                 }
                 __syncthreads();
@@ -718,7 +760,7 @@ static moe_status launch_decode_bits(DecodeArgs a, cudaStream_t stream, cudaEven
 }
 
 moe_status run_decode_layer(const uint16_t *x, int64_t T, int64_t H, int64_t I, int32_t k,
-                            int32_t bits, const moe_expert *experts, const moe_expert *shared,
+                            int32_t bits, const moe_expert *experts, int32_t n_experts, const moe_expert *shared,
                             const int32_t *unique, const int32_t *n_unique, const int32_t *offsets,
                             const int32_t *tok, const int32_t *pos, const int32_t *idx,
                             const float *w, float *h, float *yp, int32_t *tile_cnt, float *y,
@@ -746,6 +788,7 @@ moe_status run_decode_layer(const uint16_t *x, int64_t T, int64_t H, int64_t I, 
     a.tile_cnt = tile_cnt;
     a.accumulate = accumulate;
     a.flags = flags;
+    a.n_experts = n_experts;
     const bool tg1 = T == 1;
     switch (bits) {
     case 4: return tg1 ? launch_decode_bits<4, 1>(a, stream, ev_down) : launch_decode_bits<4, 2>(a, stream, ev_down);

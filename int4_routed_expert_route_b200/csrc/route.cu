@@ -208,8 +208,9 @@ __global__ void __launch_bounds__(SEL_WARPS * 32) route_select(SelArgs a) {
 // Decode-size batches (T <= 8): logits, selection and batch-union bucketing in
 // one launch.  Every block computes one expert's logits; the last block to
 // finish (ticket counter in the workspace header) routes the tokens with all
-// its threads (block-parallel ranks) and then buckets the (token, slot) pairs
-// with a stable counting sort.
+// its threads (select_tokens) and then, for two or more tokens, buckets the
+// (token, slot) pairs with a stable counting sort (one token's slots are its
+// segments as they are).
 // The counter is reset by that block for the next call.
 // ---------------------------------------------------------------------------
 constexpr int FUSED_MAXT = 8;
@@ -327,8 +328,12 @@ __global__ void __launch_bounds__(RL_WARPS * 32) route_fused_small(FusedRouteArg
     int32_t *idx_s = reinterpret_cast<int32_t *>(scratch + T * select_scratch_words(E, k, ng, tkg));  // [T][k]
     select_tokens<BlockBar>(s_all, b_all, static_cast<int>(T), E, k, ng, tkg, a.sel.rsf, a.sel.topp, scratch,
                             idx_s, a.sel.w_out, threadIdx.x, blockDim.x);
-    bucket_tiny(idx_s, a.sel.idx_out, static_cast<int>(T * k), k, E, a.counts, a.offsets, a.list, a.tok,
-                a.pos, a.unique, a.n_unique, a.flags, reinterpret_cast<int *>(dsm));
+    if (T == 1) {  // one token: the GEMV kernels read the selection slots directly
+        for (int p = threadIdx.x; p < k; p += blockDim.x) a.sel.idx_out[p] = idx_s[p];
+    } else {
+        bucket_tiny(idx_s, a.sel.idx_out, static_cast<int>(T * k), k, E, a.counts, a.offsets, a.list, a.tok,
+                    a.pos, a.unique, a.n_unique, a.flags, reinterpret_cast<int *>(dsm));
+    }
     for (int i = threadIdx.x; i < a.n_zero; i += blockDim.x) a.zero_cnt[i] = 0;
     if (threadIdx.x == 0) *a.counter = 0u;
 }
