@@ -130,6 +130,19 @@ MOE_API moe_status moe_workspace_init(void *ws, size_t ws_bytes, cudaStream_t st
 MOE_API moe_status moe_workspace_status(const void *ws, cudaStream_t stream, uint32_t *flags_out);
 
 /*
+ * Bound every on-chip wait of the calls that use `ws` to wait_us microseconds
+ * (0: the default of two seconds), async on stream.  The kernels that wait on
+ * one another's progress inside a launch (the tensor-core passes, the fused
+ * decode kernel) give up a wait after that long, latch MOE_FLAG_WAIT_TIMEOUT
+ * and return with their results invalid; waits that drain copies or
+ * tensor-core work already in flight keep the two-second bound.  The value is
+ * stored in the workspace header, so moe_workspace_init resets it to the
+ * default.  Errors: MOE_ERR_WORKSPACE if ws is NULL, misaligned or smaller
+ * than 4 KiB; MOE_ERR_CUDA if the write cannot be queued.
+ */
+MOE_API moe_status moe_workspace_set_wait_limit(void *ws, size_t ws_bytes, uint32_t wait_us, cudaStream_t stream);
+
+/*
  * Per-row symmetric quantisation and packing (load time).
  * Source: "Show HN", implemented features (per-row scales, packed int4/int2,
  * int8); ideipro.ru item (packing checked bit for bit).  For each row r:

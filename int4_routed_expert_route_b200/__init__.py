@@ -30,7 +30,7 @@ EXPORTS = ["moe_status_str", "moe_abi_version", "moe_workspace_init", "moe_works
            "moe_layer_forward", "moe_layer_forward_ex", "moe_rmsnorm_bf16",
            "moe_stack_workspace_bytes", "moe_stack_forward",
            "moe_route_noalloc_max_scratch_bytes", "moe_route_topk_noalloc",
-           "moe_layer_workspace_bytes_ex"]
+           "moe_layer_workspace_bytes_ex", "moe_workspace_set_wait_limit"]
 
 
 class MoEError(RuntimeError):
@@ -93,6 +93,7 @@ def load():
         getattr(L, name).restype = ctypes.c_int
     L.moe_workspace_init.argtypes = [_vp, _sz, _vp]
     L.moe_workspace_status.argtypes = [_vp, _vp, ctypes.POINTER(ctypes.c_uint32)]
+    L.moe_workspace_set_wait_limit.argtypes = [_vp, _sz, ctypes.c_uint32, _vp]
     L.moe_quantize_rows.argtypes = [_vp, _i64, _i64, _i32, _vp, _vp, _vp]
     L.moe_route_topk.argtypes = [_vp, _i64, _i64, _vp, _vp, ctypes.POINTER(moe_router_cfg), _vp,
                                  _vp, _vp, _vp, _sz, _vp]
@@ -166,6 +167,12 @@ class Workspace:
     def reset(self):
         _check("moe_workspace_init", load().moe_workspace_init(_ptr(self.buf), self.nbytes,
                                                               _stream()))
+
+    def set_wait_limit(self, wait_us, stream=None):
+        """Bound the on-chip waits of calls on this workspace (0: two seconds)."""
+        _check("moe_workspace_set_wait_limit",
+               load().moe_workspace_set_wait_limit(_ptr(self.buf), self.nbytes, int(wait_us),
+                                                   _stream(stream)))
 
 
 # ----------------------------------------------------------------------------- quantise

@@ -57,7 +57,8 @@ moe_status run_gemv_single(const uint16_t *x, int64_t T, int64_t H, int64_t I, c
                            float *y, uint32_t *flags, cudaStream_t stream);
 
 static constexpr size_t kAlign = 256;
-// Workspace header of a layer call: flag word at 0, router ticket at 64, down
+// Workspace header of a layer call: flag word at 0, router ticket at 64, wait
+// bound at 72 (kHdrWaitWord), tensor-path counters at 128, down
 // tile-completion counters at 1024 (zeroed by moe_workspace_init).
 static constexpr size_t kHeaderBytes = 4096;
 static size_t up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
@@ -137,6 +138,10 @@ void record_stage_event(cudaEvent_t ev, cudaStream_t s) {
 
 }  // namespace moe
 
+namespace moe {
+__global__ void set_header_word(uint32_t *word, uint32_t value) { *word = value; }
+}  // namespace moe
+
 using namespace moe;
 
 #define CUDA_OK(x) ((x) == cudaSuccess)
@@ -170,6 +175,13 @@ moe_status moe_workspace_status(const void *ws, cudaStream_t stream, uint32_t *f
     if (!CUDA_OK(cudaMemcpy(&f, ws, sizeof(f), cudaMemcpyDeviceToHost))) return MOE_ERR_CUDA;
     if (flags_out) *flags_out = f;
     return f ? MOE_ERR_DEVICE_FLAG : MOE_OK;
+}
+
+moe_status moe_workspace_set_wait_limit(void *ws, size_t ws_bytes, uint32_t wait_us, cudaStream_t stream) {
+    if (!ws || ws_bytes < kHeaderBytes || !aligned16(ws)) return MOE_ERR_WORKSPACE;
+    uint32_t *word = static_cast<uint32_t *>(ws) + kHdrWaitWord;
+    set_header_word<<<1, 1, 0, stream>>>(word, wait_us);
+    return CUDA_OK(cudaGetLastError()) ? MOE_OK : MOE_ERR_CUDA;
 }
 
 moe_status moe_quantize_rows(const float *w, int64_t rows, int64_t cols, int32_t bits,

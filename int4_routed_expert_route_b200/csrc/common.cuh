@@ -21,6 +21,17 @@ __device__ __forceinline__ void raise_flag(uint32_t *flags, uint32_t bit) {
     if (flags) atomicOr(flags, bit);
 }
 
+// Header word 18 (bytes 72..75 of a workspace): the bound, in microseconds, of
+// every on-chip wait in the kernels that have any (0: two seconds).  Waits that
+// drain copies or tensor-core work still in flight before a block exits keep the
+// full two-second bound whatever it says.
+constexpr int kHdrWaitWord = 18;
+constexpr uint64_t kFullWaitNs = 2000000000ull;
+__device__ __forceinline__ uint64_t wait_limit_ns(const uint32_t *hdr) {
+    const uint32_t us = hdr ? *const_cast<const volatile uint32_t *>(hdr + kHdrWaitWord) : 0u;
+    return us ? static_cast<uint64_t>(us) * 1000ull : kFullWaitNs;
+}
+
 // ----------------------------------------------------------------------------
 // Small arithmetic helpers.
 // ----------------------------------------------------------------------------

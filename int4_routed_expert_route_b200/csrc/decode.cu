@@ -69,7 +69,7 @@ constexpr int MAXE = 256;
 // Workspace header words (the header is zeroed by moe_workspace_init).
 constexpr int HW_ROUTE = 16;   // router blocks that have published their scores
 constexpr int HW_EXIT = 17;    // blocks that have finished
-constexpr int HW_WAIT_US = 18; // bound of every wait in microseconds (0: 2 s)
+constexpr int HW_WAIT_US = kHdrWaitWord; // bound of every wait in microseconds (0: 2 s)
 constexpr int HW_GU = 32;      // blocks that have finished every gate/up row
 constexpr int HW_TILES = 256;  // [<= 768] down rows finished per 64-row tile of H
 
@@ -358,10 +358,17 @@ __device__ __forceinline__ void stage_copy(Smem &S, int n, const void *const *sr
         mbar_expect(bar, tot);
         for (int i = 0; i < n; i++) bulk_g2s_plain(smem_u32(dst[i]), src[i], bytes[i], bar);
     }
-    bool ok = true;
-    if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, ph & 1u, c);
-    ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-    (void)ok;  // on a timeout the block has aborted; the contents are not used for anything valid
+    if ((threadIdx.x & 31) == 0 && !mbar_wait(bar, ph & 1u, c)) {
+        // the block has aborted and uses the contents for nothing valid, but the
+        // copies must land before the buffer is refilled or the block exits:
+        // drain with the full two-second bound
+        Ctl dr = c;
+        dr.limit_ns = kFullWaitNs;
+        volatile int never = 0;
+        dr.abort = &never;
+        mbar_wait(bar, ph & 1u, dr);
+    }
+    __syncwarp();
     ph++;
 }
 
@@ -1168,7 +1175,7 @@ __global__ void __launch_bounds__(THREADS, 1) decode_layer(Args a) {
     const int T = a.T;
     const uint32_t wus = a.hdr[HW_WAIT_US];
     Ctl c;
-    c.limit_ns = wus ? static_cast<uint64_t>(wus) * 1000ull : 2000000000ull;
+    c.limit_ns = wus ? static_cast<uint64_t>(wus) * 1000ull : kFullWaitNs;
     c.abort = &S.abort;
     c.flags = a.hdr;
 
@@ -1215,7 +1222,7 @@ __global__ void __launch_bounds__(THREADS, 1) decode_layer(Args a) {
             // drain: no bulk copy may still be writing this block's shared
             // memory when it exits (this wait keeps the full two-second bound)
             Ctl dr = c;
-            dr.limit_ns = 2000000000ull;
+            dr.limit_ns = kFullWaitNs;
             volatile int never = 0;
             dr.abort = &never;
             const uint32_t first = issued_end > NST ? issued_end - NST : 0;

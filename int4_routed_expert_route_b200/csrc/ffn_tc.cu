@@ -31,8 +31,10 @@
 // Tensor memory (512 columns): pass 1 = gate and up accumulators (2 x 192) +
 // two A stages of 2 x 32 columns; pass 2 = two accumulators (2 x 192, so the
 // epilogue of one tile overlaps the MMAs of the next) + four A stages of 32.
-// Hand-offs use mbarriers only; every wait is bounded and a timeout latches
-// MOE_FLAG_WAIT_TIMEOUT, stops the CTA and frees its tensor memory.
+// Hand-offs use mbarriers only; every wait is bounded (by the workspace's wait
+// bound, two seconds by default) and a timeout latches MOE_FLAG_WAIT_TIMEOUT and
+// stops the CTA: its TMA loads and MMAs in flight are drained with the full
+// two-second bound, then it frees its tensor memory and returns.
 #include <cstring>
 
 #include <cuda.h>
@@ -121,23 +123,24 @@ __device__ __forceinline__ uint64_t global_ns() {
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
     return t;
 }
-// Bounded wait on a barrier phase: false once about two seconds have passed
-// (or after 2^30 polls, whichever comes first).
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+// Bounded wait on a barrier phase: false once limit_ns have passed (the
+// workspace's wait bound for waits on other warps' progress, kFullWaitNs for the
+// drains before exit), or after 2^30 polls, whichever comes first.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
     if (mbar_try(bar, parity)) return true;
     const uint64_t t0 = global_ns();
-    for (uint32_t it = 0; it < (1u << 22); it++) {
-        for (int i = 0; i < 256; i++)
+    for (uint32_t it = 0; it < (1u << 28); it++) {
+        for (int i = 0; i < 4; i++)
             if (mbar_try(bar, parity)) return true;
-        if (global_ns() - t0 > 2000000000ull) return false;
+        if (global_ns() - t0 > limit_ns) return false;
     }
     return false;
 }
 
 // Warp-wide bounded wait: lane 0 polls, the other lanes take its verdict.
-__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, int lane) {
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, int lane, uint64_t limit_ns) {
     bool ok = true;
-    if (lane == 0) ok = mbar_wait(bar, parity);
+    if (lane == 0) ok = mbar_wait(bar, parity, limit_ns);
     return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
 }
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
@@ -388,6 +391,7 @@ __global__ void __launch_bounds__(THREADS, 1) tc_ffn(const __grid_constant__ TcM
     tc_fence_after();
     const uint32_t tmem = misc[0];
     volatile uint32_t *abort_flag = &misc[1];
+    const uint64_t lim = wait_limit_ns(a.flags);  // waits on the other warps' progress
 
     const int64_t total_chunks = static_cast<int64_t>(a.n_shared_chunks) + a.tile_off[a.E];
     const int64_t ntiles = total_chunks * mtiles;
@@ -411,7 +415,7 @@ __global__ void __launch_bounds__(THREADS, 1) tc_ffn(const __grid_constant__ TcM
                 bool ok = true;
                 for (int kt = 0; kt < KT; kt++) {
                     const uint32_t slot = kc % SB;
-                    if (!mbar_wait(B_EMPTY + 8 * slot, ((kc / SB) & 1) ^ 1)) {
+                    if (!mbar_wait(B_EMPTY + 8 * slot, ((kc / SB) & 1) ^ 1, lim)) {
                         fail();
                         ok = false;
                         break;
@@ -425,8 +429,10 @@ __global__ void __launch_bounds__(THREADS, 1) tc_ffn(const __grid_constant__ TcM
                 if (!ok) break;
             }
             // drain: the last load issued into each slot has landed before exit
+            // (full bound: the loads need nothing but memory)
             for (uint32_t j = kc > SB ? kc - SB : 0; j < kc; j++)
-                if (!mbar_wait(B_FULL + 8 * (j % SB), (j / SB) & 1)) raise_flag(a.flags, MOE_FLAG_WAIT_TIMEOUT);
+                if (!mbar_wait(B_FULL + 8 * (j % SB), (j / SB) & 1, kFullWaitNs))
+                    raise_flag(a.flags, MOE_FLAG_WAIT_TIMEOUT);
         }
         __syncwarp();
     } else if (warp == 1) {
@@ -447,7 +453,7 @@ __global__ void __launch_bounds__(THREADS, 1) tc_ffn(const __grid_constant__ TcM
                 const uint32_t idesc = f16_idesc(fmt, static_cast<uint32_t>(ti.npad));
                 const uint32_t ab = tc % NACC;
                 const uint32_t dbase = tmem + ab * NMAT * NT;
-                if (!mbar_wait(ACC_EMPTY + 8 * ab, ((tc / NACC) & 1) ^ 1)) {
+                if (!mbar_wait(ACC_EMPTY + 8 * ab, ((tc / NACC) & 1) ^ 1, lim)) {
                     fail();
                     break;
                 }
@@ -459,7 +465,7 @@ __global__ void __launch_bounds__(THREADS, 1) tc_ffn(const __grid_constant__ TcM
                         for (int u = 0; u < 4; u++) {
                             const uint32_t as = u % SA;
                             const uint32_t pa = SA == 4 ? pb : static_cast<uint32_t>((u >> 1) & 1);
-                            if (!mbar_wait(A_FULL + 8 * as, pa) || !mbar_wait(B_FULL + 8 * u, pb)) {
+                            if (!mbar_wait(A_FULL + 8 * as, pa, lim) || !mbar_wait(B_FULL + 8 * u, pb, lim)) {
                                 fail();
                                 ok = false;
                                 break;
@@ -481,7 +487,8 @@ __global__ void __launch_bounds__(THREADS, 1) tc_ffn(const __grid_constant__ TcM
                     // generic path (k-step counts that are not a multiple of 4)
                     for (int kt = 0; kt < KT; kt++, kc++) {
                         const uint32_t bs = kc % SB, as = kc % SA;
-                        if (!mbar_wait(A_FULL + 8 * as, (kc / SA) & 1) || !mbar_wait(B_FULL + 8 * bs, (kc / SB) & 1)) {
+                        if (!mbar_wait(A_FULL + 8 * as, (kc / SA) & 1, lim) ||
+                            !mbar_wait(B_FULL + 8 * bs, (kc / SB) & 1, lim)) {
                             fail();
                             ok = false;
                             break;
@@ -504,8 +511,9 @@ __global__ void __launch_bounds__(THREADS, 1) tc_ffn(const __grid_constant__ TcM
                 tc++;
             }
             // every MMA this thread issued has completed before the TMEM is freed
+            // (full bound: issued MMAs need nothing from the other warps)
             mma_commit(FIN);
-            if (!mbar_wait(FIN, 0)) raise_flag(a.flags, MOE_FLAG_WAIT_TIMEOUT);
+            if (!mbar_wait(FIN, 0, kFullWaitNs)) raise_flag(a.flags, MOE_FLAG_WAIT_TIMEOUT);
         }
         __syncwarp();
     } else if (warp < 10) {
@@ -572,7 +580,7 @@ __global__ void __launch_bounds__(THREADS, 1) tc_ffn(const __grid_constant__ TcM
                 }
                 const uint32_t as = kc % SA;
                 // one lane polls, the warp follows; one arrival per warp
-                if (!warp_wait(A_EMPTY + 8 * as, ((kc / SA) & 1) ^ 1, lane)) fail();
+                if (!warp_wait(A_EMPTY + 8 * as, ((kc / SA) & 1) ^ 1, lane, lim)) fail();
                 tc_fence_after();
                 const uint32_t col = L::a_col + as * L::a_stage_cols + grp * CB;
                 if constexpr (CB == 32) tmem_st32(tmem + lane_bits + col, v);
@@ -593,7 +601,7 @@ __global__ void __launch_bounds__(THREADS, 1) tc_ffn(const __grid_constant__ TcM
             const TileInfo ti = tile_info<PASS>(a, tile, mtiles, R, K);
             if (!ti.ok) continue;
             const uint32_t ab = tc % NACC;
-            if (!warp_wait(ACC_FULL + 8 * ab, (tc / NACC) & 1, lane)) fail();
+            if (!warp_wait(ACC_FULL + 8 * ab, (tc / NACC) & 1, lane, lim)) fail();
             tc_fence_after();
             const Tile &t = ti.t;
             const int row = t.m0 + r;
