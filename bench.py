@@ -8,7 +8,8 @@ gate/up + SwiGLU, down projection, combine.  Weight quantisation is load time
 and is reported separately.
 
 Timing: W warm-up steps, then K timed steps; L2 (126 MB) is flushed before each
-step by writing a 256 MB buffer outside the timed events; each step is timed
+step by writing a 256 MB buffer and reading it back (so the lines the step
+evicts are clean) outside the timed events; each step is timed
 with CUDA events on the launching stream; the job time is the max over ranks.
 With --gpus N > 1 every rank runs its own replica (the layer does not shard:
 no collective on the data path), so scaling is weak.
@@ -167,11 +168,19 @@ def job_tokens_per_s(tokens_per_step, steps, world, max_ms):
     return tokens_per_step * steps * world / (max_ms * 1e-3)
 
 
+# Profiling captures only (--alias-experts N): quantise N experts and let the
+# router's E slots alias them, for a small device footprint under ncu.  The
+# kernels stream the same bytes per step (8 routed experts hit 8 slots; two slots
+# aliasing one expert are still read twice), but timed numbers are not taken so.
+ALIAS_EXPERTS = 0
+
+
 def build_layer(cfg, layer=0, dev="cuda"):
     experts = []
     t0 = time.perf_counter()
     qbytes = 0
-    for e in range(cfg.E + 1):
+    n_real = cfg.E if not ALIAS_EXPERTS else min(ALIAS_EXPERTS, cfg.E)
+    for e in list(range(n_real)) + [cfg.E]:
         w = [syn.expert_weight(cfg, layer, e, m, dev) for m in ("gate", "up", "down")]
         ex = lib.QuantExpert.from_fp32(*w, bits=cfg.bits)
         qbytes += sum(x.numel() * 4 for x in w)
@@ -179,8 +188,8 @@ def build_layer(cfg, layer=0, dev="cuda"):
         del w
     torch.cuda.synchronize()
     load_s = time.perf_counter() - t0
-    table = lib.ExpertTable(experts[:cfg.E], dev)
-    shared = lib.SharedExpert(experts[cfg.E], dev)
+    table = lib.ExpertTable([experts[e % n_real] for e in range(cfg.E)], dev)
+    shared = lib.SharedExpert(experts[n_real], dev)
     gate = syn.router_gate(cfg, layer, dev)
     bias = syn.router_bias(cfg, layer, dev)
     rc = lib.router_cfg(cfg.E, cfg.k, cfg.n_group, cfg.topk_group, cfg.rsf, cfg.topp)
@@ -232,6 +241,15 @@ def workload_name(cfg):
 
 
 
+def flush_l2(buf, i):
+    """Evict L2 before a step: write the 256 MB buffer (twice L2), then read it
+    back, so that the lines the step evicts are clean (a decode loop evicts the
+    previous layer's weights, which are clean too) and no write-back of the
+    flush itself lands inside the timed step."""
+    buf.fill_(i & 0xff)
+    buf.view(torch.int64).sum()
+
+
 def _staged_steps(L, bias, xs, cfg, T, flush, dev):
     """Per-step device times of moe_layer_forward over the steps in xs [n, T, H]
     (L2 flushed before each step, outside the events), replayed from one
@@ -247,7 +265,7 @@ def _staged_steps(L, bias, xs, cfg, T, flush, dev):
         e.record(stream)
 
     def step(i):
-        flush.fill_(i & 0xff)
+        flush_l2(flush, i)
         lib.moe_layer_forward(xs[i], L["gate"], bias, rc, L["table"], L["shared"], cfg.bits, y=y,
                               ws=ws, events=ev[i], idx_out=idx[i])
 
@@ -340,19 +358,19 @@ def run_ours(args, world, rank):
     # the same steps with every stage event gives the stage breakdown and the
     # dominant kernel's duration.
     for i in range(W):
-        flush.fill_(i & 0xff)
+        flush_l2(flush, i)
         step(i, ev[i])
     torch.cuda.synchronize()
     ends = [[ev[i][0]] + [None] * (lib.LAYER_EVENTS - 2) + [ev[i][-1]] for i in range(nsteps)]
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph):
         for i in range(W, nsteps):
-            flush.fill_(i & 0xff)
+            flush_l2(flush, i)
             step(i, ends[i])
     staged = torch.cuda.CUDAGraph()
     with torch.cuda.graph(staged):
         for i in range(W, nsteps):
-            flush.fill_(i & 0xff)
+            flush_l2(flush, i)
             step(i, ev[i])
     torch.cuda.synchronize()
     staged.replay()
@@ -381,7 +399,7 @@ def run_ours(args, world, rank):
     e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
               for _ in range(nsteps)]
     for i in range(nsteps):
-        flush.fill_(i & 0xff)
+        flush_l2(flush, i)
         e2e_ev[i][0].record(stream)
         dx.copy_(hx[i], non_blocking=True)
         lib.moe_layer_forward(dx, L["gate"], L["bias"], L["rc"], L["table"], L["shared"],
@@ -450,7 +468,7 @@ def run_ours(args, world, rank):
         "dtype_detail": DTYPE_DETAIL[1 if T <= 2 else (2 if T <= 8 else 3)],
         "data": "synthetic (seeded N(0,0.02) weights quantised on device; x ~ N(0,1) bf16)",
         "config": {"workload": workload_name(cfg), "tokens_per_step": T,
-                   "l2": "flushed before every step (256 MB write, outside the timed events)",
+                   "l2": "flushed before every step (256 MB write, then read back so the evicted lines are clean; outside the timed events)",
                    "parallelism": f"replicas x{world}"},
         "expert_gbs": round(float(np.mean(expert_bytes_step)) / (total_ms / K * 1e-3) / 1e9, 1),
         "expert_bytes_per_step": int(np.mean(expert_bytes_step)),
@@ -502,13 +520,13 @@ def run_stack(args, world, rank):
         lib.moe_stack_forward(resid[i], params, rc, I, eps=1e-6, idx_out=idx[i], ws=ws)
 
     for i in range(W):
-        flush.fill_(i & 0xff)
+        flush_l2(flush, i)
         step(i)
     torch.cuda.synchronize()
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph):
         for i in range(W, nsteps):
-            flush.fill_(i & 0xff)
+            flush_l2(flush, i)
             ev[i][0].record()  # the capturing stream
             step(i)
             ev[i][1].record()
@@ -532,7 +550,7 @@ def run_stack(args, world, rank):
     dr = torch.empty((T, H), dtype=torch.float32, device=dev)
     e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(nsteps)]
     for i in range(nsteps):
-        flush.fill_(i & 0xff)
+        flush_l2(flush, i)
         e2e_ev[i][0].record(stream)
         dr.copy_(hr[i], non_blocking=True)
         lib.moe_stack_forward(dr, params, rc, I, eps=1e-6, ws=ws)
@@ -565,7 +583,7 @@ def run_stack(args, world, rank):
         "config": {"workload": f"{cfg.name}: {nl} layers, T={T} per step, H={H} I={I} E={cfg.E}+1 "
                                f"shared top-{cfg.k}, RMSNorm eps 1e-6 + fp32 residual",
                    "tokens_per_step": T,
-                   "l2": "flushed before every step (256 MB write) and the step streams "
+                   "l2": "flushed before every step (256 MB write, then read back) and the step streams "
                          f"{float(np.mean(bytes_step)) / 1e9:.1f} GB",
                    "parallelism": f"replicas x{world}"},
         "expert_gbs": round(achieved, 1),
@@ -683,7 +701,12 @@ def main():
                     help="skip the small-batch and prefill numbers of the decode workload")
     ap.add_argument("--repeat", type=int, default=10,
                     help="replays of the captured timed loop (the last one is reported)")
+    ap.add_argument("--alias-experts", type=int, default=0,
+                    help="profiling captures only: quantise this many experts and alias the "
+                         "router's slots onto them (small device footprint)")
     args = ap.parse_args()
+    global ALIAS_EXPERTS
+    ALIAS_EXPERTS = args.alias_experts
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":
@@ -696,6 +719,8 @@ def main():
     world, rank, _ = dist_setup()
     res = run_stack(args, world, rank) if args.workload in STACKS else run_ours(args, world, rank)
     if rank == 0:
+        if ALIAS_EXPERTS:
+            res["config"]["alias_experts"] = f"{ALIAS_EXPERTS} (profiling capture; not a benchmark number)"
         print(json.dumps(res))
     if world > 1:
         torch.distributed.destroy_process_group()
