@@ -250,8 +250,10 @@ MOE_API moe_status moe_expert_ffn(const uint16_t *x, int64_t T, int64_t H, int64
  *   y       [T, H] fp32, overwritten
  *   idx_out [T, k] int32 and w_out [T, k] fp32, nullable (routing decision)
  * ws: moe_layer_workspace_bytes(T, H, I, cfg) bytes.
- * Paths (AUTO): one or two tokens run a fused router + bucketing launch and two
- * streaming GEMV launches; 3..8 tokens run one persistent kernel (router,
+ * Paths (AUTO): one or two tokens run a fused router launch (logits, selection
+ * and, for two tokens, bucketing; one token's k slots are its segments as they
+ * are) and two streaming GEMV launches (int4 dot products as exact int32 dp4a
+ * sums per lane chunk); 3..8 tokens run one persistent kernel (router,
  * selection, gate/up, down and combine, every expert's rows split evenly over
  * all SMs, exact integer dot products); from 9 tokens on, int4 layers run the
  * tcgen05 tensor-core grouped GEMM (int4 codes converted to bf16 / fp16 in

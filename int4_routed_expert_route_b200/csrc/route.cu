@@ -326,8 +326,10 @@ __global__ void __launch_bounds__(RL_WARPS * 32) route_fused_small(FusedRouteArg
     const int ng = a.sel.n_group, tkg = a.sel.topk_group, k = a.sel.k;
     float *scratch = b_all + T * E;
     int32_t *idx_s = reinterpret_cast<int32_t *>(scratch + T * select_scratch_words(E, k, ng, tkg));  // [T][k]
+    float *w_s = reinterpret_cast<float *>(idx_s + T * k);  // [T][k]: the top-p ranking reads it back
     select_tokens<BlockBar>(s_all, b_all, static_cast<int>(T), E, k, ng, tkg, a.sel.rsf, a.sel.topp, scratch,
-                            idx_s, a.sel.w_out, threadIdx.x, blockDim.x);
+                            idx_s, w_s, threadIdx.x, blockDim.x);
+    for (int p = threadIdx.x; p < T * k; p += blockDim.x) a.sel.w_out[p] = w_s[p];
     if (T == 1) {  // one token: the GEMV kernels read the selection slots directly
         for (int p = threadIdx.x; p < k; p += blockDim.x) a.sel.idx_out[p] = idx_s[p];
     } else {
@@ -416,9 +418,9 @@ moe_status launch_route_fused(const uint16_t *x, int64_t T, int64_t H, const flo
     a.zero_cnt = zero_cnt;
     a.n_zero = n_zero;
     const int E = cfg->n_experts;
-    // scores, biased scores, the selection's scratch and the selected indices
+    // scores, biased scores, the selection's scratch and the selected indices and weights
     size_t smem = static_cast<size_t>(
-                      2 * T * E + T * (select_scratch_words(E, cfg->top_k, cfg->n_group, cfg->topk_group) + cfg->top_k)) *
+                      2 * T * E + T * (select_scratch_words(E, cfg->top_k, cfg->n_group, cfg->topk_group) + 2 * cfg->top_k)) *
                   sizeof(float);
     const size_t bsm = static_cast<size_t>(2 * T * cfg->top_k) * sizeof(int);  // bucket_tiny
     if (bsm > smem) smem = bsm;

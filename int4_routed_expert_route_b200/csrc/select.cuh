@@ -190,6 +190,40 @@ static __device__ void select_core(const SelArgs &a, int64_t t, const float *s_s
     else select_core_j<32>(a, t, s_sm, b_sm, pick);
 }
 
+// Expert top-p of one token by its warp, the same decisions as finish_weights:
+// lane r < k holds slot r's index and weight.  The total is summed in slot
+// order and the running sum in rank order (descending weight, ties to the lower
+// slot), each as one sequential fp32 chain that every lane repeats, so the
+// roundings are finish_weights' own; the slot of rank i is kept when i = 0 or
+// the sum of ranks below i is still short of topp * total.  Dropped slots get
+// index -1 and weight 0.  A handful of shuffles instead of one lane's k^2 loop.
+static __device__ __forceinline__ void topp_warp(int k, float topp, int lane, int &idx, float &w) {
+    float total = 0.0f;
+    for (int j = 0; j < k; j++) total += __shfl_sync(0xffffffffu, w, j);
+    int rank = 0;
+    for (int j = 0; j < k; j++) {
+        const float o = __shfl_sync(0xffffffffu, w, j);
+        rank += (o > w) || (o == w && j < lane);
+    }
+    float by_rank = 0.0f;  // lane i: the weight of rank i
+    for (int j = 0; j < k; j++) {
+        const float o = __shfl_sync(0xffffffffu, w, j);
+        if (__shfl_sync(0xffffffffu, rank, j) == lane) by_rank = o;
+    }
+    const float target = topp * total;
+    float run = 0.0f, before = 0.0f;
+    for (int i = 0; i < k; i++) {
+        if (lane == i) before = run;
+        run += __shfl_sync(0xffffffffu, by_rank, i);
+    }
+    const bool keep_rank = lane == 0 || before < target;  // for rank = lane
+    const bool keep = __shfl_sync(0xffffffffu, keep_rank ? 1 : 0, lane < k ? rank : 0) != 0;
+    if (lane < k && !keep) {
+        idx = -1;
+        w = 0.0f;
+    }
+}
+
 // Block-parallel group-limited top-k of T tokens from their scores s_all and
 // biased scores b_all ([T][E] in shared memory), by nthr threads at once (a
 // multiple of 32; Bar::sync() joins them): every (token, expert) finds its rank
@@ -199,7 +233,7 @@ static __device__ void select_core(const SelArgs &a, int64_t t, const float *s_s
 // (descending biased score, ties to the lower expert; four adjacent lanes split
 // the comparisons): rank r < k is slot r.  Then the weights (finish_weights'
 // arithmetic, one warp per token with the sum in slot order).  The same order
-// and tie rules as select_core.  scratch holds T * (3 n_group + topk_group + k)
+// and tie rules as select_core (top-p by topp_warp).  scratch holds T * (3 n_group + topk_group + k)
 // words; idx_out / w_out [T][k] may be shared or global memory.
 template <class Bar>
 static __device__ __forceinline__ void select_block_ranks(const float *s_all, const float *b_all, int T, int E,
@@ -277,12 +311,13 @@ static __device__ __forceinline__ void select_block_ranks(const float *s_all, co
             const int po = __shfl_sync(0xffffffffu, pr, r);
             if (po >= 0) sum += o;
         }
+        int id = pr;
+        float wv = pr >= 0 ? (sv / sum) * rsf : 0.0f;
+        if (topp > 0.0f && topp < 1.0f) topp_warp(k, topp, lane, id, wv);
         if (lane < k) {
-            idx_out[t * k + lane] = pr;
-            w_out[t * k + lane] = pr >= 0 ? (sv / sum) * rsf : 0.0f;
+            idx_out[t * k + lane] = id;
+            w_out[t * k + lane] = wv;
         }
-        __syncwarp();
-        if (topp > 0.0f && topp < 1.0f && lane == 0) finish_weights(st, pk, k, rsf, topp, idx_out + t * k, w_out + t * k);
     }
     Bar::sync();
 }
@@ -403,13 +438,13 @@ static __device__ __forceinline__ void select_block_warps(const float *s_all, co
             const float o = __shfl_sync(0xffffffffu, sv, r);
             if (__shfl_sync(0xffffffffu, mine, r) >= 0) sum += o;
         }
+        int id = mine;
+        float wv = mine >= 0 ? (sv / sum) * rsf : 0.0f;
+        if (topp > 0.0f && topp < 1.0f) topp_warp(k, topp, lane, id, wv);
         if (lane < k) {
-            idx_out[t * k + lane] = mine;
-            w_out[t * k + lane] = mine >= 0 ? (sv / sum) * rsf : 0.0f;
+            idx_out[t * k + lane] = id;
+            w_out[t * k + lane] = wv;
         }
-        __syncwarp();
-        if (topp > 0.0f && topp < 1.0f && lane == 0)
-            finish_weights(st, pick + t * k, k, rsf, topp, idx_out + t * k, w_out + t * k);
     }
     Bar::sync();
 }
