@@ -129,6 +129,10 @@ __device__ __forceinline__ f2 f2_sub(f2 a, f2 b) {
 }
 
 __device__ __forceinline__ float silu(float g) { return g / (1.0f + expf(-g)); }
+// SiLU with the hardware exponential and reciprocal (a few ulp of fp32): for h
+// that is rounded to fp16 right after (relative 2^-11), where expf and an IEEE
+// division only cost issue slots.
+__device__ __forceinline__ float silu_fast(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
 
 // 128-bit streaming load that does not allocate in L1 (weights are read once).
 __device__ __forceinline__ uint4 ldg_stream(const void *p) {

@@ -55,7 +55,6 @@ constexpr int THREADS = 448;  // producer, MMA, 8 converter warps, 4 epilogue wa
 constexpr int NCONV = 256;    // converter threads
 constexpr int NEPI = 128;     // epilogue threads (= TMEM lanes)
 constexpr int SB = 4;         // token-tile ring depth
-constexpr int SC = 8;         // per-thread code ring depth (prefetch SC-1 steps)
 
 constexpr int BTILE_BYTES = NT * BK * 2;    // 24 KB: 192 rows x 128 B
 constexpr int BOX_BYTES = BOX * BK * 2;     // 8 KB
@@ -69,6 +68,7 @@ struct Smem {
     static constexpr uint32_t tmem_cols = 512;
     static_assert(a_col + SA * a_stage_cols <= tmem_cols, "tensor memory budget");
     static constexpr int CB = NMAT == 2 ? 32 : 16;   // code bytes (= A columns) per converter thread per k-step
+    static constexpr int SC = 8;   // per-thread code ring depth (prefetch SC-1 k-steps; 12 / 16 measured no faster)
     static_assert(2 * CB == static_cast<int>(a_stage_cols), "two converter groups fill one A stage");
     static constexpr size_t b_off = 0;                                               // [SB][BTILE]
     static constexpr size_t c_off = b_off + static_cast<size_t>(SB) * BTILE_BYTES;   // [SC][CB/16][NCONV][16]
@@ -215,18 +215,26 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t *r) {
 }
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
+// K order of the tensor-core operands.  Within every group of 8 consecutive
+// K indices (one 32-bit word of codes) the MMA's K positions 2m and 2m + 1 hold
+// the columns m and m + 4 (m = 0..3): a code pair at nibbles m and m + 4 sits at
+// bits 4m and 4m + 16 of the word, so one shift and one LOP3 put it into both
+// halves of a 16-bit pair.  The B operands are stored in the same order (the
+// gathered x rows of pass 1, the h rows written by pass 1's epilogue), so every
+// product meets its own activation.
+__device__ __forceinline__ int k_slot(int col) {  // MMA K position of column col
+    const int q = col & 7;
+    return (col & ~7) | (q < 4 ? 2 * q : 2 * q - 7);
+}
+
 // 8 int4 codes (one 32-bit word, consecutive columns) -> 8 16-bit values q
-// (exact), as 4 words of value pairs.  magic = bit pattern of 16-bit 128 (bf16)
-// or 1024 (fp16) in both halves; sub = the pattern of magic + 8.
+// (exact) in the K order above, as 4 words of value pairs (m, m + 4).
+// magic = bit pattern of 16-bit 128 (bf16) or 1024 (fp16) in both halves;
+// sub = the pattern of magic + 8.
 __device__ __forceinline__ uint4 codes_to_16bit(uint32_t v, uint32_t magic, uint32_t sub) {
-    const uint32_t lo = v & 0x0F0F0F0Fu;         // even columns, one per byte
-    const uint32_t hi = (v >> 4) & 0x0F0F0F0Fu;  // odd columns
     uint32_t o[4];
 #pragma unroll
-    for (int m = 0; m < 4; m++) {
-        const uint32_t p = __byte_perm(lo, hi, static_cast<uint32_t>(m | ((4 + m) << 8)));
-        o[m] = (p & 0x00FF00FFu) | magic;
-    }
+    for (int m = 0; m < 4; m++) o[m] = ((v >> (4 * m)) & 0x000F000Fu) | magic;
     uint4 r;
     if (magic == 0x43004300u) {
         asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(r.x) : "r"(o[0]), "r"(sub));
@@ -342,7 +350,7 @@ template <int PASS>
 __global__ void __launch_bounds__(THREADS, 1) tc_ffn(const __grid_constant__ TcMaps maps, TcArgs a) {
     constexpr int NMAT = PASS == 1 ? 2 : 1;
     using L = Smem<NMAT>;
-    constexpr int NACC = L::NACC, SA = L::SA, CB = L::CB;
+    constexpr int NACC = L::NACC, SA = L::SA, CB = L::CB, SC = L::SC;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *b_tiles = sm + L::b_off;
@@ -609,7 +617,7 @@ __global__ void __launch_bounds__(THREADS, 1) tc_ffn(const __grid_constant__ TcM
             if (!aborted()) {
                 if (PASS == 1) {
                     const float sg = t.ex->gate.scale[row], su = t.ex->up.scale[row];
-                    __half *hp = a.h + (t.hrow + t.j0) * a.I + row;
+                    __half *hp = a.h + (t.hrow + t.j0) * a.I + k_slot(row);  // pass 2's K order
                     bool ovf = false;
                     for (int c0 = 0; c0 < ti.npad; c0 += 32) {
                         uint32_t g[32], u[32];
@@ -621,7 +629,7 @@ __global__ void __launch_bounds__(THREADS, 1) tc_ffn(const __grid_constant__ TcM
                             if (j < t.n) {
                                 const float gv = __uint_as_float(g[i]) * sg;
                                 const float uv = __uint_as_float(u[i]) * su;
-                                const float hv = silu(gv) * uv;
+                                const float hv = silu_fast(gv) * uv;
                                 ovf |= !(fabsf(hv) <= 65504.0f);
                                 hp[static_cast<int64_t>(j) * a.I] = __float2half_rn(hv);
                             }
@@ -655,15 +663,27 @@ __global__ void __launch_bounds__(THREADS, 1) tc_ffn(const __grid_constant__ TcM
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(L::tmem_cols) : "memory");
 }
 
-// Rows of x in expert-sorted order: xs[q] = x[tok[q]] for the routed pairs.
+// Pass 1's B rows in the MMA's K order (k_slot): xs[q] = x[tok[q]] for the
+// routed pairs q < n_rows (of cap rows), then xs[cap + t] = x[t] for the shared
+// expert's T rows.  A 16-byte vector is one group of 8 columns (c0..c7) and
+// becomes (c0, c4, c1, c5, c2, c6, c3, c7).
 __global__ void gather_rows(const uint16_t *__restrict__ x, const int32_t *__restrict__ tok,
-                            const int32_t *__restrict__ n_rows, int64_t H, uint16_t *__restrict__ xs) {
+                            const int32_t *__restrict__ n_rows, int64_t cap, int64_t T_shared, int64_t H,
+                            uint16_t *__restrict__ xs) {
     const int64_t n = *n_rows;
     const int64_t per = H / 8;  // 16-byte vectors per row
-    for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n * per;
+    for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < (cap + T_shared) * per;
          i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
         const int64_t q = i / per, v = i % per;
-        reinterpret_cast<uint4 *>(xs + q * H)[v] = reinterpret_cast<const uint4 *>(x + static_cast<int64_t>(tok[q]) * H)[v];
+        if (q < cap && q >= n) continue;
+        const int64_t src = q < cap ? static_cast<int64_t>(tok[q]) : q - cap;
+        const uint4 w = reinterpret_cast<const uint4 *>(x + src * H)[v];
+        uint4 o;
+        o.x = __byte_perm(w.x, w.z, 0x5410);
+        o.y = __byte_perm(w.x, w.z, 0x7632);
+        o.z = __byte_perm(w.y, w.w, 0x5410);
+        o.w = __byte_perm(w.y, w.w, 0x7632);
+        reinterpret_cast<uint4 *>(xs + q * H)[v] = o;
     }
 }
 
@@ -677,7 +697,7 @@ bool tc_ok(int64_t H, int64_t I) {
 }
 
 size_t tc_xs_bytes(int64_t T, int32_t k, int64_t H) {
-    return static_cast<size_t>(T * k) * static_cast<size_t>(H) * sizeof(uint16_t);
+    return static_cast<size_t>(T * k + T) * static_cast<size_t>(H) * sizeof(uint16_t);
 }
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
@@ -743,19 +763,22 @@ moe_status run_tc_layer(const uint16_t *x, int64_t T, int64_t H, int64_t I, int3
     a.yp = yp;
     a.w = w;
     a.bits = 4;
-    // expert-sorted copy of x for the TMA loads of pass 1
+    // expert-sorted copy of x (and the shared expert's copy) in the MMA's K
+    // order, for the TMA loads of pass 1
+    const int64_t t_sh = shared ? T : 0;
+    uint16_t *xs16 = static_cast<uint16_t *>(xs);
     {
-        const int64_t vecs = T * k * (H / 8);
+        const int64_t vecs = (T * k + t_sh) * (H / 8);
         int64_t grid = (vecs + 255) / 256;
         if (grid > 65535) grid = 65535;
         if (grid > 0) {
-            gather_rows<<<static_cast<unsigned>(grid), 256, 0, stream>>>(x, tok, offsets + E, H,
-                                                                         static_cast<uint16_t *>(xs));
+            gather_rows<<<static_cast<unsigned>(grid), 256, 0, stream>>>(x, tok, offsets + E, T * k, t_sh, H, xs16);
             if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
         }
     }
     TcMaps m1, m2;
-    if (!make_map(&m1.b_main, xs, T * k, H, true) || !make_map(&m1.b_shared, x, T, H, true) ||
+    if (!make_map(&m1.b_main, xs16, T * k, H, true) ||
+        !make_map(&m1.b_shared, xs16 + T * k * H, t_sh > 0 ? t_sh : T, H, true) ||
         !make_map(&m2.b_main, h, T * k + T, I, false))
         return MOE_ERR_CUDA;
     m2.b_shared = m2.b_main;
