@@ -456,16 +456,16 @@ static __host__ __device__ __forceinline__ int select_scratch_words(int E, int k
 }
 
 // Group-limited top-k of T tokens by nthr threads (Bar::sync() joins them):
-// from three tokens on the warp-reduction form where the configuration fits it
-// and has at most 16 groups (about three times faster than the rank form at
-// eight tokens of 256 experts in 8 groups), else the rank form (the faster of
-// the two for one or two tokens, and with many small groups).
+// from two tokens on the warp-reduction form where the configuration fits it
+// and has at most 16 groups (1.3 times faster than the rank form at two tokens
+// of 256 experts in 8 groups, three times at eight), else the rank form (the
+// faster of the two for one token, and with many small groups).
 // scratch: T * select_scratch_words() words.
 template <class Bar>
 static __device__ __forceinline__ void select_tokens(const float *s_all, const float *b_all, int T, int E, int k,
                                                      int ng, int tkg, float rsf, float topp, float *scratch,
                                                      int32_t *idx_out, float *w_out, int tid, int nthr) {
-    if (T >= 3 && ng <= 16 && select_warps_fit(E, k, ng, tkg))
+    if (T >= 2 && ng <= 16 && select_warps_fit(E, k, ng, tkg))
         select_block_warps<Bar>(s_all, b_all, T, E, k, ng, tkg, rsf, topp, scratch, idx_out, w_out, tid, nthr);
     else
         select_block_ranks<Bar>(s_all, b_all, T, E, k, ng, tkg, rsf, topp, scratch, idx_out, w_out, tid, nthr);
