@@ -13,7 +13,7 @@
 // int4 codes are exact in bf16 and fp16, so dequantising to 16 bits adds no
 // error; the row scale is applied in the epilogue in fp32.
 //
-// Warp roles (448 threads, one CTA per SM):
+// Warp roles (pass 1: 576 threads, pass 2: 448; one CTA per SM):
 //   warp 0     TMA producer: per k-step, 2D tiled loads of 64-row boxes bring the
 //              tile's token rows x 64 columns of the B operand into the K-major
 //              128B-swizzled layout (pass 1 reads the expert-sorted copy of x,
@@ -26,8 +26,10 @@
 //              16-bit values in registers ahead of time, and writes them into
 //              the A stage in tensor memory (tcgen05.st) once the MMA has
 //              released that stage
-//   warps 10-13 epilogue: after a tile's last MMA, read the accumulator lanes
-//              (tcgen05.ld), apply row scales, SwiGLU (pass 1) and store
+//   warps 10-  epilogue (pass 1: 8 warps, two per lane quarter taking alternate
+//              32-column chunks; pass 2: 4): after a tile's last MMA, read the
+//              accumulator lanes (tcgen05.ld), apply row scales, SwiGLU (pass 1)
+//              and store
 // Tensor memory (512 columns): pass 1 = gate and up accumulators (2 x 192) +
 // two A stages of 2 x 32 columns; pass 2 = two accumulators (2 x 192, so the
 // epilogue of one tile overlaps the MMAs of the next) + four A stages of 32.
@@ -51,9 +53,11 @@ constexpr int BM = 128;       // weight rows per tile (MMA M)
 constexpr int BK = 64;        // columns per k-step (one 128-byte swizzle row)
 constexpr int NT = 192;       // max tokens per tile (MMA N)
 constexpr int BOX = 64;       // token rows per TMA box
-constexpr int THREADS = 448;  // producer, MMA, 8 converter warps, 4 epilogue warps
+// producer, MMA, 8 converter warps, then the epilogue warps: pass 1 (SwiGLU on
+// two accumulators, one of them to drain before the next tile) 8, pass 2 4
+constexpr int threads_of(int pass) { return pass == 1 ? 576 : 448; }
 constexpr int NCONV = 256;    // converter threads
-constexpr int NEPI = 128;     // epilogue threads (= TMEM lanes)
+constexpr int nepi_of(int pass) { return threads_of(pass) - 320; }  // epilogue threads
 constexpr int SB = 4;         // token-tile ring depth
 
 constexpr int BTILE_BYTES = NT * BK * 2;    // 24 KB: 192 rows x 128 B
@@ -347,7 +351,7 @@ __device__ __forceinline__ TileInfo tile_info(const TcArgs &a, int64_t tile, int
 // The warp-specialized persistent grouped-GEMM kernel.
 // ---------------------------------------------------------------------------
 template <int PASS>
-__global__ void __launch_bounds__(THREADS, 1) tc_ffn(const __grid_constant__ TcMaps maps, TcArgs a) {
+__global__ void __launch_bounds__(threads_of(PASS), 1) tc_ffn(const __grid_constant__ TcMaps maps, TcArgs a) {
     constexpr int NMAT = PASS == 1 ? 2 : 1;
     using L = Smem<NMAT>;
     constexpr int NACC = L::NACC, SA = L::SA, CB = L::CB, SC = L::SC;
@@ -383,7 +387,7 @@ __global__ void __launch_bounds__(THREADS, 1) tc_ffn(const __grid_constant__ TcM
         }
         for (int i = 0; i < NACC; i++) {
             mbar_init(ACC_FULL + 8 * i, 1);
-            mbar_init(ACC_EMPTY + 8 * i, NEPI / 32);  // one arrival per epilogue warp
+            mbar_init(ACC_EMPTY + 8 * i, nepi_of(PASS) / 32);  // one arrival per epilogue warp
         }
         mbar_init(FIN, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -603,6 +607,8 @@ __global__ void __launch_bounds__(THREADS, 1) tc_ffn(const __grid_constant__ TcM
     } else {
         // ---------------- epilogue ----------------
         const int quarter = warp & 3;                  // TMEM lane quarter this warp may read
+        constexpr int CSTEP = nepi_of(PASS) / 4;      // two warps per lane quarter in pass 1: alternate chunks
+        const int c_first = ((warp - 10) >> 2) * 32;   // this warp's 32-column chunks: c_first, + CSTEP, ...
         const int r = quarter * 32 + lane;             // weight row within the tile
         uint32_t tc = 0;
         for (int64_t tile = blockIdx.x; tile < ntiles && !aborted(); tile += gridDim.x) {
@@ -619,7 +625,7 @@ __global__ void __launch_bounds__(THREADS, 1) tc_ffn(const __grid_constant__ TcM
                     const float sg = t.ex->gate.scale[row], su = t.ex->up.scale[row];
                     __half *hp = a.h + (t.hrow + t.j0) * a.I + k_slot(row);  // pass 2's K order
                     bool ovf = false;
-                    for (int c0 = 0; c0 < ti.npad; c0 += 32) {
+                    for (int c0 = c_first; c0 < ti.npad; c0 += CSTEP) {
                         uint32_t g[32], u[32];
                         tmem_ld32(lane_addr + c0, g);
                         tmem_ld32(lane_addr + NT + c0, u);
@@ -639,7 +645,7 @@ __global__ void __launch_bounds__(THREADS, 1) tc_ffn(const __grid_constant__ TcM
                 } else {
                     const float sd = t.ex->down.scale[row];
                     float *yq = a.yp + (t.hrow + t.j0) * a.H + row;
-                    for (int c0 = 0; c0 < ti.npad; c0 += 32) {
+                    for (int c0 = c_first; c0 < ti.npad; c0 += CSTEP) {
                         uint32_t d[32];
                         tmem_ld32(lane_addr + c0, d);
 #pragma unroll
@@ -786,7 +792,7 @@ moe_status run_tc_layer(const uint16_t *x, int64_t T, int64_t H, int64_t I, int3
         const size_t smem = Smem<2>::total;
         if (cudaFuncSetAttribute(tc_ffn<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess)
             return MOE_ERR_CUDA;
-        tc_ffn<1><<<sms, THREADS, smem, stream>>>(m1, a);
+        tc_ffn<1><<<sms, threads_of(1), smem, stream>>>(m1, a);
         if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
     }
     if (ev_down) record_stage_event(ev_down, stream);
@@ -794,7 +800,7 @@ moe_status run_tc_layer(const uint16_t *x, int64_t T, int64_t H, int64_t I, int3
         const size_t smem = Smem<1>::total;
         if (cudaFuncSetAttribute(tc_ffn<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess)
             return MOE_ERR_CUDA;
-        tc_ffn<2><<<sms, THREADS, smem, stream>>>(m2, a);
+        tc_ffn<2><<<sms, threads_of(2), smem, stream>>>(m2, a);
         if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
     }
     return MOE_OK;
