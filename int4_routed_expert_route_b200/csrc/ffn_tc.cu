@@ -221,9 +221,10 @@ __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.
 
 // K order of the tensor-core operands.  Within every group of 8 consecutive
 // K indices (one 32-bit word of codes) the MMA's K positions 2m and 2m + 1 hold
-// the columns m and m + 4 (m = 0..3): a code pair at nibbles m and m + 4 sits at
-// bits 4m and 4m + 16 of the word, so one shift and one LOP3 put it into both
-// halves of a 16-bit pair.  The B operands are stored in the same order (the
+// the columns m and m + 4 (m = 0..3): once the word's even and odd nibbles are
+// spread over bytes (two masks), such a pair sits in bytes 0 and 2 or 1 and 3
+// of one of the two words, and one byte permute with the magic's high byte
+// makes the 16-bit pair.  The B operands are stored in the same order (the
 // gathered x rows of pass 1, the h rows written by pass 1's epilogue), so every
 // product meets its own activation.
 __device__ __forceinline__ int k_slot(int col) {  // MMA K position of column col
@@ -236,9 +237,14 @@ __device__ __forceinline__ int k_slot(int col) {  // MMA K position of column co
 // magic = bit pattern of 16-bit 128 (bf16) or 1024 (fp16) in both halves;
 // sub = the pattern of magic + 8.
 __device__ __forceinline__ uint4 codes_to_16bit(uint32_t v, uint32_t magic, uint32_t sub) {
+    const uint32_t even = v & 0x0F0F0F0Fu;         // bytes: nibbles 0, 2, 4, 6
+    const uint32_t odd = (v >> 4) & 0x0F0F0F0Fu;   // bytes: nibbles 1, 3, 5, 7
+    const uint32_t hi = (magic >> 8 & 0xFFu) * 0x01010101u;  // the magic's high byte, four times
     uint32_t o[4];
-#pragma unroll
-    for (int m = 0; m < 4; m++) o[m] = ((v >> (4 * m)) & 0x000F000Fu) | magic;
+    o[0] = __byte_perm(even, hi, 0x4240);  // nibbles 0, 4
+    o[1] = __byte_perm(odd, hi, 0x4240);   // 1, 5
+    o[2] = __byte_perm(even, hi, 0x4341);  // 2, 6
+    o[3] = __byte_perm(odd, hi, 0x4341);   // 3, 7
     uint4 r;
     if (magic == 0x43004300u) {
         asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(r.x) : "r"(o[0]), "r"(sub));
