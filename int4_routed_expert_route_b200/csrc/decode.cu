@@ -497,6 +497,10 @@ __device__ void produce_phase(const Args &a, Smem &S, const Phase &P, int item_b
             const int s = static_cast<int>(st % NST);
             bool go = !*c.abort;
             if (go && st >= NST) go = mbar_wait(smem_u32(&S.empty[s]), ((st / NST) - 1) & 1, c);
+            // a consumer that gave up on a stage releases it with its copy possibly
+            // still in flight, and only after it has set abort: look again, so that
+            // no copy is ever queued into a buffer that may still be written
+            if (go) go = !*c.abort;
             if (!go) {
                 st++;
                 continue;  // aborted: issue nothing more

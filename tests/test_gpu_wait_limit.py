@@ -10,8 +10,9 @@ moe_workspace_init (which restores the default bound) the same workspace gives
 the oracle's answer again.
 
 The fused decode kernel reads the same bound but is not driven into a timeout
-here: its consumers can release a ring stage whose copy an aborted wait never
-saw land, and that path has not been shown to keep every copy accounted for."""
+here: its abort path (consumers releasing stages whose copies an aborted wait
+never saw land, the producer queueing nothing more once it sees the abort, the
+exit drain) is checked by reading only."""
 import numpy as np
 import pytest
 import torch
