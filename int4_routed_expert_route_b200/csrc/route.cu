@@ -99,7 +99,10 @@ __global__ void __launch_bounds__(RL_WARPS * 32) route_logits_small(const uint16
 // ---------------------------------------------------------------------------
 // Logits for large batches: a 64-token x 64-expert tile per block, K in chunks
 // of 32.  Each thread owns 4x4 outputs; products are chained in fp32 over one
-// 32-wide chunk and the chunk sums are accumulated in fp64.
+// 32-wide chunk and the chunk sums are accumulated in fp64.  The chunks are
+// double-buffered in shared memory: the next chunk's global loads are in
+// flight while the current one is multiplied (H is a multiple of 64, so every
+// chunk is full).
 // ---------------------------------------------------------------------------
 constexpr int RT_T = 64, RT_E = 64, RT_K = 32;
 
@@ -107,44 +110,63 @@ __global__ void __launch_bounds__(256) route_logits_tiled(const uint16_t *__rest
                                                           int64_t T, int64_t H,
                                                           const float *__restrict__ G, int E,
                                                           float *__restrict__ logits) {
-    __shared__ float xs[RT_K][RT_T + 4];
-    __shared__ float gs[RT_K][RT_E + 4];
+    __shared__ float xs[2][RT_K][RT_T + 4];
+    __shared__ float gs[2][RT_K][RT_E + 4];
     const int tid = threadIdx.x;
     const int ty = tid / 16, tx = tid % 16;
     const int64_t t0 = static_cast<int64_t>(blockIdx.x) * RT_T;
     const int e0 = blockIdx.y * RT_E;
+    // this thread's share of a chunk: 8 bf16 of one token (16 B), 2 x 4 fp32 of the gate
+    const int xt = tid / 4, xk = (tid % 4) * 8;
+    const bool x_in = t0 + xt < T;
+    const uint16_t *xrow = x + (x_in ? t0 + xt : 0) * H + xk;
+    int g_e[2], g_k[2];
+    bool g_in[2];
+    const float *grow[2];
+#pragma unroll
+    for (int r = 0; r < 2; r++) {
+        const int idx = tid + 256 * r;
+        g_e[r] = idx / 8;
+        g_k[r] = (idx % 8) * 4;
+        g_in[r] = e0 + g_e[r] < E;
+        grow[r] = G + static_cast<int64_t>(g_in[r] ? e0 + g_e[r] : 0) * H + g_k[r];
+    }
+    uint4 xv_r;
+    float4 gv_r[2];
+    auto load_chunk = [&](int64_t kc) {
+        xv_r = x_in ? *reinterpret_cast<const uint4 *>(xrow + kc) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+        for (int r = 0; r < 2; r++)
+            gv_r[r] = g_in[r] ? *reinterpret_cast<const float4 *>(grow[r] + kc) : make_float4(0.f, 0.f, 0.f, 0.f);
+    };
+    auto store_chunk = [&](int b) {
+        const uint32_t w4[4] = {xv_r.x, xv_r.y, xv_r.z, xv_r.w};
+#pragma unroll
+        for (int i = 0; i < 4; i++) {
+            xs[b][xk + 2 * i][xt] = bf16_bits_to_float(w4[i] & 0xffffu);
+            xs[b][xk + 2 * i + 1][xt] = bf16_bits_to_float(w4[i] >> 16);
+        }
+#pragma unroll
+        for (int r = 0; r < 2; r++) {
+            gs[b][g_k[r]][g_e[r]] = gv_r[r].x;
+            gs[b][g_k[r] + 1][g_e[r]] = gv_r[r].y;
+            gs[b][g_k[r] + 2][g_e[r]] = gv_r[r].z;
+            gs[b][g_k[r] + 3][g_e[r]] = gv_r[r].w;
+        }
+    };
     double dacc[4][4];
 #pragma unroll
     for (int i = 0; i < 4; i++)
 #pragma unroll
         for (int j = 0; j < 4; j++) dacc[i][j] = 0.0;
 
-    for (int64_t kc = 0; kc < H; kc += RT_K) {
-        {   // x tile: 64 tokens x 32 bf16; thread loads 8 bf16 (16 B)
-            const int tt = tid / 4, kk = (tid % 4) * 8;
-            uint4 v = make_uint4(0, 0, 0, 0);
-            if (t0 + tt < T) v = *reinterpret_cast<const uint4 *>(x + (t0 + tt) * H + kc + kk);
-            const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-            for (int i = 0; i < 4; i++) {
-                xs[kk + 2 * i][tt] = bf16_bits_to_float(w4[i] & 0xffffu);
-                xs[kk + 2 * i + 1][tt] = bf16_bits_to_float(w4[i] >> 16);
-            }
-        }
-        {   // gate tile: 64 experts x 32 fp32; thread loads 2 float4
-#pragma unroll
-            for (int r = 0; r < 2; r++) {
-                const int idx = tid + 256 * r;
-                const int ee = idx / 8, kk = (idx % 8) * 4;
-                float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (e0 + ee < E) v = *reinterpret_cast<const float4 *>(G + static_cast<int64_t>(e0 + ee) * H + kc + kk);
-                gs[kk][ee] = v.x;
-                gs[kk + 1][ee] = v.y;
-                gs[kk + 2][ee] = v.z;
-                gs[kk + 3][ee] = v.w;
-            }
-        }
-        __syncthreads();
+    const int64_t nchunks = H / RT_K;
+    load_chunk(0);
+    store_chunk(0);
+    __syncthreads();
+    for (int64_t c = 0; c < nchunks; c++) {
+        const int b = static_cast<int>(c & 1);
+        if (c + 1 < nchunks) load_chunk((c + 1) * RT_K);
         float facc[4][4];
 #pragma unroll
         for (int i = 0; i < 4; i++)
@@ -152,8 +174,8 @@ __global__ void __launch_bounds__(256) route_logits_tiled(const uint16_t *__rest
             for (int j = 0; j < 4; j++) facc[i][j] = 0.0f;
 #pragma unroll 8
         for (int kk = 0; kk < RT_K; kk++) {
-            const float4 xv = *reinterpret_cast<const float4 *>(&xs[kk][ty * 4]);
-            const float4 gv = *reinterpret_cast<const float4 *>(&gs[kk][tx * 4]);
+            const float4 xv = *reinterpret_cast<const float4 *>(&xs[b][kk][ty * 4]);
+            const float4 gv = *reinterpret_cast<const float4 *>(&gs[b][kk][tx * 4]);
             const float xa[4] = {xv.x, xv.y, xv.z, xv.w};
             const float ga[4] = {gv.x, gv.y, gv.z, gv.w};
 #pragma unroll
@@ -165,6 +187,8 @@ __global__ void __launch_bounds__(256) route_logits_tiled(const uint16_t *__rest
         for (int i = 0; i < 4; i++)
 #pragma unroll
             for (int j = 0; j < 4; j++) dacc[i][j] += static_cast<double>(facc[i][j]);
+        // the other buffer was last read before the previous barrier
+        if (c + 1 < nchunks) store_chunk(b ^ 1);
         __syncthreads();
     }
 #pragma unroll
