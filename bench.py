@@ -287,7 +287,7 @@ def _staged_steps(L, bias, xs, cfg, T, flush, dev):
 
 
 def secondary_numbers(L, cfg, flush, dev, peaks, peak_kind, steps=8):
-    """Small batches with the Zipf-skewed router (T = 2, 8, 32) and the
+    """Small batches with the Zipf-skewed router (T = 2, 4, 8, 32) and the
     4096-token prefill, on the same resident experts as the headline."""
     H, I = cfg.H, cfg.I
     ex_bytes = 2 * (I * H // 2 + I * 4) + (H * I // 2 + H * 4)
@@ -295,7 +295,7 @@ def secondary_numbers(L, cfg, flush, dev, peaks, peak_kind, steps=8):
                    "per-step CUDA events, medians over the steps"}
     zipf = syn.router_bias(syn.SMALL_BATCH, 0, dev)
     small = {}
-    for T in (2, 8, 32):
+    for T in (2, 4, 8, 32):
         xs = syn.activations(steps * T, H, 7001 + T, dev).view(steps, T, H)
         step_ms, _, idx = _staged_steps(L, zipf, xs, cfg, T, flush, dev)
         uniq = np.array([len(np.unique(r[r >= 0])) for r in idx])

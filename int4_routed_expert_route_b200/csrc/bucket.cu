@@ -3,10 +3,14 @@
 // batch is streamed once and applied to all of its positions ("Show HN: running
 // GLM 5.2 on a slow computer", implemented features, batch-union MoE).
 //
-// One 1024-thread block: a shared-memory histogram, a block scan, then the
-// pairs in chunks of 1024 in pair order; inside a chunk the rank of a pair
-// among equal experts comes from __match_any_sync within the warp plus a
-// per-warp count table scanned across warps, which keeps the sort stable.
+// One 1024-thread block.  Warp w owns the contiguous pair range
+// [w P / 32, (w + 1) P / 32) and counts its pairs per expert (ranks among equal
+// experts of one 32-pair step come from __match_any_sync); one pass over the
+// experts turns the 32 per-warp counts into exclusive prefixes in warp order
+// and the experts' totals into offsets; each warp then walks its range again
+// and places its pairs.  Pairs of earlier warps, earlier steps and lower lanes
+// come first, which keeps the sort stable; there are four block barriers in
+// all, independent of the batch size.
 #include "common.cuh"
 
 namespace moe {
@@ -23,29 +27,54 @@ struct BucketArgs {
     int32_t *tile_off;  // [E+1] exclusive prefix of ceil(count / ntile)
 };
 
+constexpr int BK_WARPS = BK_THREADS / 32;
+constexpr int BK_BATCH = 8;  // 32-pair steps whose indices are loaded together
+
 __global__ void __launch_bounds__(BK_THREADS) bucket_kernel(BucketArgs a) {
     extern __shared__ int sm[];
     const int E = a.E;
-    int *cnt = sm;                    // [E] counts, then cursors
-    int *ctot = sm + E;               // [E] chunk totals
-    int *wtot = sm + 2 * E;           // [33] scan scratch
-    uint16_t *wcnt = reinterpret_cast<uint16_t *>(sm + 2 * E + 40);  // [32][E]
+    int *wc = sm;                        // [32][E] per-warp counts, then per-warp cursors
+    int *base = sm + BK_WARPS * E;       // [E] offsets
+    int *wtot = sm + (BK_WARPS + 1) * E; // [33] scan scratch
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    const int64_t r0 = a.P * wid / BK_WARPS, r1 = a.P * (wid + 1) / BK_WARPS;
+    int *mine = wc + wid * E;
 
-    for (int e = tid; e < E; e += BK_THREADS) cnt[e] = 0;
+    for (int i = tid; i < BK_WARPS * E; i += BK_THREADS) wc[i] = 0;
     __syncthreads();
+    // 1. per-warp counts over the warp's range
     bool bad = false;
-    for (int64_t p = tid; p < a.P; p += BK_THREADS) {
-        const int e = a.idx[p];
-        if (e >= E) bad = true;
-        else if (e >= 0) atomicAdd(&cnt[e], 1);
+    for (int64_t b0 = r0; b0 < r1; b0 += 32 * BK_BATCH) {
+        int ev[BK_BATCH];
+#pragma unroll
+        for (int j = 0; j < BK_BATCH; j++) {
+            const int64_t p = b0 + 32 * j + lane;
+            ev[j] = p < r1 ? a.idx[p] : -1;
+        }
+#pragma unroll
+        for (int j = 0; j < BK_BATCH; j++) {
+            const int e = ev[j];
+            if (e >= E) bad = true;
+            const bool valid = e >= 0 && e < E;
+            const unsigned m = __match_any_sync(0xffffffffu, valid ? e : -1);
+            if (valid && (__ffs(m) - 1) == lane) mine[e] += __popc(m);
+            __syncwarp();
+        }
     }
     if (__syncthreads_or(bad) && tid == 0) raise_flag(a.flags, MOE_FLAG_BAD_EXPERT_INDEX);
 
-    // offsets, unique list, tile table (E <= 1024: one expert per thread)
+    // 2. per expert (one per thread, E <= 1024): exclusive prefixes over the
+    //    warps, then offsets, the unique list and the tile table
     {
         const int e = tid;
-        const int c = e < E ? cnt[e] : 0;
+        int c = 0;
+        if (e < E) {
+            for (int w = 0; w < BK_WARPS; w++) {
+                const int v = wc[w * E + e];
+                wc[w * E + e] = c;
+                c += v;
+            }
+        }
         int tot;
         const int off = block_exclusive_scan(c, wtot, &tot);
         const int nz = (c > 0) ? 1 : 0;
@@ -60,7 +89,7 @@ __global__ void __launch_bounds__(BK_THREADS) bucket_kernel(BucketArgs a) {
             a.offsets[e] = off;
             if (nz) a.unique[upos] = e;
             if (a.tile_off) a.tile_off[e] = toff;
-            cnt[e] = off;  // becomes the cursor
+            base[e] = off;
         }
         if (tid == 0) {
             a.offsets[E] = tot;
@@ -70,45 +99,36 @@ __global__ void __launch_bounds__(BK_THREADS) bucket_kernel(BucketArgs a) {
     }
     __syncthreads();
 
-    for (int64_t base = 0; base < a.P; base += BK_THREADS) {
-        for (int i = tid; i < 32 * E; i += BK_THREADS) wcnt[i] = 0;
-        __syncthreads();
-        const int64_t p = base + tid;
-        const int e = (p < a.P) ? a.idx[p] : -1;
-        const bool valid = (e >= 0 && e < E);
-        const int key = valid ? e : -1;
-        const unsigned mask = __match_any_sync(0xffffffffu, key);
-        const int rank = __popc(mask & lanemask_lt());
-        const bool leader = (__ffs(mask) - 1) == lane;
-        if (valid && leader) wcnt[wid * E + e] = static_cast<uint16_t>(__popc(mask));
-        __syncthreads();
-        for (int ee = tid; ee < E; ee += BK_THREADS) {
-            int run = 0;
-            for (int w = 0; w < 32; w++) {
-                const int c = wcnt[w * E + ee];
-                wcnt[w * E + ee] = static_cast<uint16_t>(run);
-                run += c;
+    // 3. each warp places its pairs, in pair order
+    for (int64_t b0 = r0; b0 < r1; b0 += 32 * BK_BATCH) {
+        int ev[BK_BATCH];
+#pragma unroll
+        for (int j = 0; j < BK_BATCH; j++) {
+            const int64_t p = b0 + 32 * j + lane;
+            ev[j] = p < r1 ? a.idx[p] : -1;
+        }
+#pragma unroll
+        for (int j = 0; j < BK_BATCH; j++) {
+            const int64_t p = b0 + 32 * j + lane;
+            const int e = ev[j];
+            const bool valid = e >= 0 && e < E;
+            const unsigned m = __match_any_sync(0xffffffffu, valid ? e : -1);
+            if (valid) {
+                const int q = base[e] + mine[e] + __popc(m & lanemask_lt());
+                a.list[q] = static_cast<int32_t>(p);
+                if (a.tok) a.tok[q] = static_cast<int32_t>(p / a.k);
+                if (a.pos) a.pos[p] = q;
+            } else if (p < r1 && a.pos) {
+                a.pos[p] = -1;
             }
-            ctot[ee] = run;
+            __syncwarp();  // every lane has read the cursor before its leader moves it
+            if (valid && (__ffs(m) - 1) == lane) mine[e] += __popc(m);
+            __syncwarp();
         }
-        __syncthreads();
-        if (valid) {
-            const int q = cnt[e] + wcnt[wid * E + e] + rank;
-            a.list[q] = static_cast<int32_t>(p);
-            if (a.tok) a.tok[q] = static_cast<int32_t>(p / a.k);
-            if (a.pos) a.pos[p] = q;
-        } else if (p < a.P && a.pos) {
-            a.pos[p] = -1;
-        }
-        __syncthreads();
-        for (int ee = tid; ee < E; ee += BK_THREADS) cnt[ee] += ctot[ee];
-        __syncthreads();
     }
 }
 
-size_t bucket_smem_bytes(int E) {
-    return static_cast<size_t>(2 * E + 40) * sizeof(int) + static_cast<size_t>(32) * E * sizeof(uint16_t);
-}
+size_t bucket_smem_bytes(int E) { return static_cast<size_t>((BK_WARPS + 1) * E + 40) * sizeof(int); }
 
 moe_status launch_bucket(const int32_t *idx, int64_t T, int32_t k, int32_t E, int32_t *counts,
                          int32_t *offsets, int32_t *list, int32_t *tok, int32_t *pos,
