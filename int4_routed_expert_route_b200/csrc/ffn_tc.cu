@@ -141,7 +141,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint64_
     return false;
 }
 
-// Warp-wide bounded wait: lane 0 polls, the other lanes take its verdict.
+// Warp-wide bounded wait: lane 0 polls, the other lanes take its result.
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, int lane, uint64_t limit_ns) {
     bool ok = true;
     if (lane == 0) ok = mbar_wait(bar, parity, limit_ns);
