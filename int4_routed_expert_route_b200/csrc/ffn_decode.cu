@@ -7,12 +7,17 @@
 //    row space; blocks split it so that each works inside one expert (blocks
 //    per expert = grid / experts), every SM streaming about the same bytes.
 //    Warp (kw, rg) owns the 16-byte chunks [32kw, 32kw+32) of the rows
-//    rg, rg+RG, ... of its range; its activation slice (pre-scaled by 2^-e,
-//    read with 16-byte loads) stays in registers.  Each lane streams its own
-//    chunks through a private cp.async ring in shared memory.
-//  - An int4 code c at bit 4p of a word is decoded as the exact float
-//    2^23 + c*2^e (one lop3 with 0x4B000000), one packed subtract and one packed
-//    FMA per pair of codes.
+//    rg, rg+RG, ... of its range; its activation slice (read with 16-byte
+//    loads) stays in registers.  Each lane streams its own chunks through a
+//    private cp.async ring in shared memory.
+//  - int4: a lane's 32 activations become integers X = round(x * 2^F) (one
+//    exponent per lane chunk, |X| < 2^22) split into three byte limbs; a code
+//    word's even and odd nibbles meet the limb words in six dp4a, the code bias
+//    enters as -8 * sum(X), and the chunk's dot product is exact in int32 and
+//    rounded once to fp32.  int8 / int2: a code c at bit p of a word is decoded
+//    as the exact float 2^23 + c*2^e (one lop3 with 0x4B000000) against
+//    activations pre-scaled by 2^-e, one packed subtract and one packed FMA per
+//    pair of codes.
 //  - Partial dot products are reduced across the warp with a reduce-scatter
 //    butterfly (V values in V-1 + log2(32/V) shuffles instead of 5V) and across
 //    the K-slice warps once per run in shared memory, in a fixed order.
