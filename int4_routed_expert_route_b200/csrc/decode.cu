@@ -11,8 +11,9 @@
 //             products summed in fp64, rounded once), the sigmoid and the biased
 //             score, and publish them; a counter tells every block when all
 //             scores are out.  Each block then runs the group-limited top-k
-//             itself (one warp per token) instead of waiting for one block to
-//             do it: no serial tail between the router and the experts.
+//             of every token itself (all its consumer threads at once,
+//             select_tokens) instead of waiting for one block to do it: no
+//             serial tail between the router and the experts.
 //   items     the (expert, token group) pairs of the batch: the shared expert's
 //             token groups first, then every unique routed expert (ascending)
 //             with its tokens in groups of TG.  A fixed set of blocks owns the

@@ -1,7 +1,10 @@
-// select.cuh -- noaux_tc group-limited top-k selection of one token by one
-// warp ("Show HN: running GLM 5.2 on a slow computer", implemented features:
-// DeepSeek-V3 style sigmoid router, noaux_tc, routed_scaling_factor).  Shared
-// by the router kernels and the fused decode-layer kernel.
+// select.cuh -- noaux_tc group-limited top-k selection ("Show HN: running GLM
+// 5.2 on a slow computer", implemented features: DeepSeek-V3 style sigmoid
+// router, noaux_tc, routed_scaling_factor), in two shapes that decide alike:
+// one token by one warp (select_core, the router's large-batch kernel) and all
+// tokens of a small batch by one block (select_tokens: the rank form at one
+// token, the warp-reduction form from two on).  Shared by the router kernels
+// and the fused decode-layer kernel.
 #pragma once
 
 #include "common.cuh"
