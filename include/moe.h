@@ -211,7 +211,8 @@ MOE_API moe_status moe_route_topk_noalloc(const uint16_t *x, int64_t T, int64_t 
  *   list    [T*k] int32: pairs of expert e at list[offsets[e] .. offsets[e+1]),
  *           in increasing p
  *   unique  [E] int32: experts with counts > 0, ascending; n_unique [1] int32
- * Needs T*k <= 2^24 and E <= 1024; no workspace (a single on-chip pass).
+ * Needs T*k <= 2^24 and E <= 1024; no workspace (one launch of one block, its
+ * counters in shared memory).
  * An index >= E latches nothing here (no ws): the call treats it as dropped;
  * moe_layer_forward checks indices itself.
  */
