@@ -1,4 +1,4 @@
-"""NumPy driver for the plain-C oracle of the routed-expert MoE layer.
+"""NumPy front end of the plain-C oracle of the routed-expert MoE layer.
 
 TEST INFRASTRUCTURE ONLY: the tests, the package smoke check and the CPU
 baseline leg of the benchmark may import this module; the product path may not.
