@@ -27,6 +27,16 @@ def test_traffic_used_only_while_sources_match(tmp_path):
     assert bench.measured_traffic("k", str(tmp_path / "missing.txt")) is None
 
 
+def test_source_hash_sees_code_not_comments():
+    # comment and layout edits keep a captured traffic figure; a code edit drops it
+    base = "int f(int a) {  // add one\n  return a + 1; /* done */\n}\n"
+    reworded = "/* header */\nint f(int a) { // increment\n\n    return a + 1;\n}"
+    changed = "int f(int a) {  // add one\n  return a + 2; /* done */\n}\n"
+    assert bench._code_only(base) == bench._code_only(reworded)
+    assert bench._code_only(base) != bench._code_only(changed)
+    assert "add one" not in bench._code_only(base)
+
+
 def test_committed_traffic_table_parses():
     # every row names existing sources and a positive byte count
     with open(os.path.join(ROOT, "profiles", "roofline_traffic.txt")) as fh:
