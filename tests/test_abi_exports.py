@@ -134,3 +134,23 @@ def test_host_side_path_and_size_contracts(so):
                                fake, need - 1, None) == 4
     assert L.moe_rmsnorm_bf16(fake, 1, 6144, ctypes.c_float(-1.0), fake, None) == 1
     assert L.moe_rmsnorm_bf16(fake, 1, 6144, ctypes.c_float(float("nan")), fake, None) == 1
+
+
+def test_bucket_limits_refused_on_host(so):
+    """moe_bucket's limits (its counters live in shared memory: E <= 1024; pair
+    indices fit 24 bits) are checked before any launch."""
+    so.moe_bucket.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32] + \
+        [ctypes.c_void_p] * 6
+    so.moe_bucket.restype = ctypes.c_int
+    f = ctypes.c_void_p(0x1000)
+
+    def call(T, k, E, idx=f, lst=f):
+        return so.moe_bucket(idx, T, k, E, f, f, lst, f, f, None)
+
+    assert call(4, 8, 1025) == 1              # more experts than shared-memory counters
+    assert call((1 << 24) // 8 + 1, 8, 256) == 1  # T * k above 2^24
+    assert call(4, 0, 256) == 1               # no slots
+    assert call(-1, 8, 256) == 1              # negative batch
+    assert call(4, 8, 256, idx=None) == 1     # pairs without indices
+    assert call(4, 8, 256, lst=None) == 1     # pairs without a list
+
